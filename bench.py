@@ -1,0 +1,451 @@
+#!/usr/bin/env python
+"""Decode-step benchmark for low-rank (per-head SVD-factored) KV-cache attention.
+
+One step = one decode step of one layer for every batch row: lrkv_append writes the
+new token's latent row per (batch row, KV head), then lrkv_decode_attn runs the
+split-KV kernel (rebuild K = Z_K B_K, V = Z_V B_V on chip, scores, online softmax,
+P V) and the log-sum-exp merge. Inputs are seeded synthetic workloads (see
+rank_kv_cache_head_b200/workloads.py) resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--algo auto|simt|tcgen05] [--impl ours|reference]
+
+Timing: the K steps are captured into CUDA graphs and replayed; the timed region is
+bracketed by a barrier and torch.cuda.synchronize on both sides and measured with
+CUDA events on the launching stream, max over ranks. The cache is rotated among
+enough copies that the bytes touched between two uses of a copy exceed 3x the L2
+size, and every copy's seqlens is restored on a parallel graph branch after its
+step, so each step attends exactly the workload's lengths. Events recorded in the
+graph around every split-kernel launch give the dominant kernel's duration.
+With --gpus N > 1 (torchrun), every rank runs its own batch (weak scaling, no
+collective on the data path) and rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import glob
+import json
+import math
+import os
+import statistics
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from rank_kv_cache_head_b200 import lrkv  # noqa: E402
+from rank_kv_cache_head_b200.metrics import (ClockSampler, max_over_ranks,  # noqa: E402
+                                             step_bytes, sum_over_ranks)
+from rank_kv_cache_head_b200.workloads import (WORKLOADS, make_append_rows,  # noqa: E402
+                                               make_inputs, seqlens_for)
+
+METRIC = "low-rank decode attention: latent GB/s, tokens/s/GPU, % of HBM roofline"
+UNIT = "GB/s"
+DEFAULT_WORKLOAD = "vlm7b-bf16"
+L2_BYTES = 126 * 1024 ** 2
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--algo", default="auto", choices=["auto", "simt", "tcgen05"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU time budget of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=100)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world <= 1:
+        return 0, 1, 0
+    import torch.distributed as dist
+    rank = int(os.environ["RANK"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "rank_kv_cache_head_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str, algo: str):
+    """DRAM bytes per split-kernel launch from the committed ncu summary, if it was
+    taken on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = j.get(f"{workload}/{algo}")
+    if not e or e.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle timing (the reference arm and the cpu_baseline field)
+# ---------------------------------------------------------------------------------------
+
+
+def oracle_sample(wl, inputs, budget_s: float, max_units=None, rng_seed=0):
+    """Time the fp64 oracle on whole (batch row, KV head) units in a seeded random
+    order until ``budget_s`` seconds of work are done. Returns (seconds per unit,
+    units timed, latent bytes timed, seconds)."""
+    from oracle import lrkv_oracle as orc
+    from rank_kv_cache_head_b200.workloads import stored_bits
+    io, lat = wl.io_dtype, wl.latent_dtype
+    q = orc.decode_stored(stored_bits(inputs["q"]), io)
+    BK = orc.decode_stored(stored_bits(inputs["BK"]), io)
+    BV = orc.decode_stored(stored_bits(inputs["BV"]), io)
+    seq = inputs["seqlens"].numpy()
+    units = [(b, g) for b in range(wl.batch) for g in range(wl.n_kv_heads)]
+    order = np.random.default_rng(rng_seed).permutation(len(units))
+    G = wl.group
+    spent, n, lat_bytes = 0.0, 0, 0
+    per_tok = 2 * wl.rank * {"f32": 4, "bf16": 2, "i8": 1, "e4m3": 1}[lat] + \
+        (8 if lat in ("i8", "e4m3") else 0)
+    for i in order:
+        b, g = units[i]
+        Lb = int(seq[b])
+        # decode this unit's stored rows (part of the oracle's work)
+        t0 = time.perf_counter()
+        ZK = orc.decode_stored(stored_bits(inputs["ZK"][b:b + 1, g:g + 1, :Lb]), lat)
+        ZV = orc.decode_stored(stored_bits(inputs["ZV"][b:b + 1, g:g + 1, :Lb]), lat)
+        SK = SV = None
+        if inputs["ZK_scale"] is not None:
+            SK = inputs["ZK_scale"][b:b + 1, g:g + 1, :Lb].numpy().astype(np.float64)
+            SV = inputs["ZV_scale"][b:b + 1, g:g + 1, :Lb].numpy().astype(np.float64)
+        orc.decode_attention(q[b:b + 1, g * G:(g + 1) * G], ZK, ZV, BK[g:g + 1], BV[g:g + 1],
+                             np.array([Lb]), SK, SV)
+        spent += time.perf_counter() - t0
+        n += 1
+        lat_bytes += Lb * per_tok
+        if spent >= budget_s or (max_units is not None and n >= max_units):
+            break
+    return spent / max(n, 1), n, lat_bytes, spent
+
+
+def run_reference(args, rank):
+    """The oracle as it stands, timed on the host cores: each step is a bounded sample
+    (one (batch row, KV head) unit, all its query heads) of the workload."""
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    target = seqlens_for(wl)
+    inputs = make_inputs(wl, capacity=int(target.max()), seqlens=target)
+    for _ in range(args.warmup):
+        oracle_sample(wl, inputs, 0.0, max_units=1, rng_seed=1)
+    times, byts = [], 0
+    for k in range(args.steps):
+        per_unit, n, lb, spent = oracle_sample(wl, inputs, 0.0, max_units=1, rng_seed=100 + k)
+        times.append(spent)
+        byts += lb
+    total = sum(times)
+    units_per_step = wl.batch * wl.n_kv_heads
+    sec_per_full_step = statistics.mean(times) * units_per_step
+    value = byts / total / 1e9
+    cores = blas_threads()
+    sample = (f"{args.steps} steps, each one (batch row, KV head) unit of {args.workload} "
+              f"({wl.group} query heads), fp64 numpy oracle, {cores} BLAS threads")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(times) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(wl, target, None, "oracle"),
+        "tokens_per_s_per_gpu": wl.batch / sec_per_full_step,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl, target, plan, algo):
+    cfg = {"workload": wl.name, "batch": wl.batch, "n_q_heads": wl.n_q_heads,
+           "n_kv_heads": wl.n_kv_heads, "d_head": wl.d_head, "rank": wl.rank,
+           "seq_len": int(target.max()) if wl.ragged_min is None else
+           f"ragged U[{wl.ragged_min},{wl.seq_len}] (mean {float(np.mean(target)):.1f})",
+           "io_dtype": wl.io_dtype, "latent_dtype": wl.latent_dtype, "kernel": algo}
+    if plan is not None:
+        cfg["plan"] = plan
+    return cfg
+
+
+# ---------------------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------------------
+
+
+def largest_divisor_at_most(k: int, cap: int) -> int:
+    for g in range(min(k, cap), 0, -1):
+        if k % g == 0:
+            return g
+    return 1
+
+
+def run_ours(args, rank, world, local):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = WORKLOADS[args.workload]
+    target = seqlens_for(wl)                         # attended lengths (after append)
+    Lmax = int(target.max())
+    capacity = ((Lmax + args.e2e_steps + 16 + 7) // 8) * 8
+    inputs = make_inputs(wl, capacity=capacity, seqlens=target)
+    sb = step_bytes(wl, target)
+    per_copy = sb["latent"] + sb["scales"]
+    n_copies = max(2, math.ceil(3 * L2_BYTES / max(per_copy, 1)))
+    n_copies = min(n_copies, 64)
+
+    dims = lrkv.make_dims(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.d_head, wl.rank, capacity,
+                          Lmax, wl.io_dtype, wl.latent_dtype, 0, args.algo)
+    plan = lrkv.plan(dims)
+    q = inputs["q"].to(dev)
+    BK, BV = inputs["BK"].to(dev), inputs["BV"].to(dev)
+    io_t = q.dtype
+    out = torch.empty_like(q)
+    ws = lrkv.new_workspace(dims, device=dev)
+    seq0 = torch.from_numpy((target - 1).astype(np.int32)).to(dev)
+    copies = []
+    for c in range(n_copies):
+        rows = make_append_rows(wl, step=c)
+        cp = {"ZK": inputs["ZK"].to(dev), "ZV": inputs["ZV"].to(dev),
+              "SK": None if inputs["ZK_scale"] is None else inputs["ZK_scale"].to(dev),
+              "SV": None if inputs["ZV_scale"] is None else inputs["ZV_scale"].to(dev),
+              "seq": seq0.clone(), "zk": rows["zk_new"].to(dev), "zv": rows["zv_new"].to(dev)}
+        cp["step"] = lrkv.PreparedStep(dims, q, cp["ZK"], cp["ZV"], cp["SK"], cp["SV"], BK, BV,
+                                       cp["seq"], out, ws, cp["zk"], cp["zv"])
+        copies.append(cp)
+    torch.cuda.synchronize()
+
+    s_main = torch.cuda.Stream(device=dev)
+    s_side = torch.cuda.Stream(device=dev)
+    # one eager step first: one-time launch set-up never happens inside a capture
+    with torch.cuda.stream(s_main):
+        copies[0]["step"](s_main.cuda_stream)
+        copies[0]["seq"].copy_(seq0)
+    torch.cuda.synchronize()
+    if lrkv.read_status(ws):
+        raise RuntimeError("device status after the first eager step")
+    G = largest_divisor_at_most(args.steps, 64)
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(G)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(G)]
+
+    def capture(nsteps, timed):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s_main):
+            cur = torch.cuda.current_stream()
+            handle = cur.cuda_stream
+            pending = {}
+            for k in range(nsteps):
+                c = k % n_copies
+                if c in pending:
+                    cur.wait_event(pending.pop(c))
+                if timed:
+                    copies[c]["step"](handle, ev_b[k].cuda_event, ev_e[k].cuda_event)
+                else:
+                    copies[c]["step"](handle)
+                done = torch.cuda.Event()
+                done.record(cur)
+                s_side.wait_event(done)
+                with torch.cuda.stream(s_side):
+                    copies[c]["seq"].copy_(seq0, non_blocking=True)
+                    rest = torch.cuda.Event()
+                    rest.record(s_side)
+                pending[c] = rest
+            for e in pending.values():
+                cur.wait_event(e)
+        return g
+
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
+    sampler = ClockSampler(gpu_id).start()
+    graph = capture(G, timed=True)
+    warm_reps = max(1, math.ceil(args.warmup / G))
+    with torch.cuda.stream(s_main):
+        for _ in range(warm_reps):
+            graph.replay()
+    torch.cuda.synchronize()
+    status = lrkv.read_status(ws)
+    if status:
+        raise RuntimeError(f"device status {status} after warm-up")
+
+    reps = args.steps // G
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    with torch.cuda.stream(s_main):
+        start.record()
+        for _ in range(reps):
+            graph.replay()
+        end.record()
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    barrier()
+    ms = start.elapsed_time(end)
+    split_ms = [ev_b[k].elapsed_time(ev_e[k]) for k in range(G)]  # last replay's launches
+    status = lrkv.read_status(ws)
+    if status:
+        raise RuntimeError(f"device status {status} after the timed region")
+    ms_max = max_over_ranks(ms, dev)
+    sampler.stop()
+    clocks = sampler.summary(t0, t1)
+
+    # ---- end to end through the public host-buffer entry point --------------------------
+    q_h = inputs["q"].pin_memory()
+    rows0 = make_append_rows(wl, step=0)
+    zk_h, zv_h = rows0["zk_new"].pin_memory(), rows0["zv_new"].pin_memory()
+    out_h = torch.empty_like(inputs["q"]).pin_memory()
+    q_d, o_d = torch.empty_like(q), torch.empty_like(q)
+    zk_d, zv_d = torch.empty_like(copies[0]["zk"]), torch.empty_like(copies[0]["zv"])
+    for cp in copies:
+        cp["seq"].copy_(seq0)
+    ke = max(1, args.e2e_steps)
+    uses = [0] * n_copies
+    e2e_lat = 0
+    for k in range(ke):
+        c = k % n_copies
+        e2e_lat += step_bytes(wl, target + uses[c])["latent"] + step_bytes(wl, target + uses[c])["scales"]
+        uses[c] += 1
+    for cp in copies:
+        cp["seq"].copy_(seq0)
+    torch.cuda.synchronize()
+    es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s_main):
+        es.record()
+        for k in range(ke):
+            cp = copies[k % n_copies]
+            lrkv.decode_step_host(dims, q_h, zk_h, zv_h, out_h, q_d, zk_d, zv_d, o_d, cp["ZK"],
+                                  cp["ZV"], cp["SK"], cp["SV"], BK, BV, cp["seq"], ws,
+                                  stream=s_main)
+            s_main.synchronize()          # the step's result is read on the host
+            _ = out_h[0, 0, 0].item()
+        ee.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(es.elapsed_time(ee), dev)
+    if lrkv.read_status(ws):
+        raise RuntimeError("device status after the end-to-end loop")
+
+    # ---- numbers -------------------------------------------------------------------------
+    peak, peak_kind = peaks()
+    lat_step = sb["latent"] + sb["scales"]
+    total_lat = sum_over_ranks(lat_step * args.steps, dev)
+    value = total_lat / (ms_max * 1e-3) / 1e9
+    split_mean_ms = statistics.mean(split_ms)
+    achieved = sb["split_kernel"] / (split_mean_ms * 1e-3) / 1e9
+    traffic = profiled_traffic(args.workload, plan["algo"])
+    e2e_value = sum_over_ranks(e2e_lat, dev) / (e2e_ms * 1e-3) / 1e9
+    io_bytes = 4 if wl.io_dtype == "f32" else 2
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": warm_reps * G, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": {"bf16": "bf16", "f32": "f32"}[wl.io_dtype] + (
+            "" if wl.latent_dtype in ("bf16", "f32") else f"+{wl.latent_dtype}-latents"),
+        "data": "synthetic (seeded; shapes and distributions of the workload definition)",
+        "config": dict(workload_config(wl, target, plan, plan["algo"]),
+                       parallelism=f"dp{world} (independent batches per GPU)",
+                       l2=f"cache rotated over {n_copies} copies ({n_copies * per_copy / 1e6:.0f} MB "
+                          f">= 3x L2) between uses"),
+        "tokens_per_s_per_gpu": wl.batch * args.steps / (ms_max * 1e-3),
+        "hbm_roofline_frac": sb["total"] * args.steps / (ms_max * 1e-3) / 1e9 / peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": f"split ({plan['algo']})", "peak_kind": peak_kind,
+                     "split_us_mean": split_mean_ms * 1e3,
+                     "bytes_per_launch": sb["split_kernel"]},
+        "e2e": {"value": e2e_value, "unit": UNIT,
+                "h2d_bytes_per_step": q.numel() * io_bytes + 2 * zk_d.numel() * io_bytes,
+                "d2h_bytes_per_step": q.numel() * io_bytes, "steps": ke,
+                "ms_per_step": e2e_ms / ke},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": None,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        per_unit, n, lb, spent = oracle_sample(wl, inputs, args.cpu_seconds)
+        cores = blas_threads()
+        cpu_val = lb / spent / 1e9
+        line["cpu_baseline"] = {
+            "value": cpu_val, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n} of {wl.batch * wl.n_kv_heads} (batch row, KV head) units, "
+                      f"{spent:.1f} s, fp64 numpy oracle",
+            "tokens_per_s": wl.batch / (per_unit * wl.batch * wl.n_kv_heads)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_init()
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank)
+        else:
+            if not torch.cuda.is_available():
+                raise SystemExit("bench.py needs a CUDA GPU for --impl ours")
+            run_ours(args, rank, world, local)
+    finally:
+        import torch.distributed as dist
+        if dist.is_available() and dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

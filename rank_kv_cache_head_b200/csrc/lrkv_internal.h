@@ -1,0 +1,83 @@
+// Internal declarations shared by the kernels and the C-ABI layer of liblrkv.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "lrkv.h"
+
+namespace lrkv {
+
+constexpr int kTile = 128;            // tokens per pipeline tile / split granule
+constexpr size_t kHeaderBytes = 256;  // workspace header: status word + counters
+
+// Workspace header words.
+enum HeaderWord { kStatusWord = 0, kWorkCounter = 1, kDoneCounter = 2 };
+
+// Launch plan for one call (depends only on dims and the device).
+struct Plan {
+  int algo;         // LRKV_ALGO_SIMT or LRKV_ALGO_TCGEN05
+  int S;            // splits per (b, KV head) at max_seqlen
+  int chunk;        // tokens per split, multiple of kTile
+  int grid;         // CTAs of the split kernel
+  int smem;         // dynamic shared memory of the split kernel
+  size_t lse_off;   // byte offset of lse partials in the workspace
+  size_t o_off;     // byte offset of o partials
+  size_t ws_bytes;  // total workspace bytes
+};
+
+// Everything the split kernels read (device pointers and sizes).
+struct SplitArgs {
+  const void* q;
+  const void* ZK;
+  const void* ZV;
+  const float* SK;
+  const float* SV;
+  const void* BK;
+  const void* BV;
+  const int32_t* seqlens;
+  float* o_part;    // [B][Hq][S][d]
+  float* lse_part;  // [B][Hq][S]
+  uint32_t* header;
+  int B, Hq, Hkv, G, d, r, Lcap, max_seqlen, S, chunk;
+  int io_dtype, latent_dtype;
+  float scale_log2;  // log2(e) / sqrt(d)
+};
+
+struct MergeArgs {
+  const float* o_part;
+  const float* lse_part;
+  const int32_t* seqlens;
+  void* out;
+  float* lse_out;
+  uint32_t* header;
+  int B, Hq, d, S, chunk, Lcap, max_seqlen;
+  int io_dtype;
+};
+
+struct AppendArgs {
+  const void* zk_new;
+  const void* zv_new;
+  void* ZK;
+  void* ZV;
+  float* SK;
+  float* SV;
+  int32_t* seqlens;
+  uint32_t* header;
+  int B, Hkv, r, Lcap;
+  int io_dtype, latent_dtype;
+};
+
+// Launchers (return a cudaError_t from the launch).
+cudaError_t launch_split_simt(const SplitArgs& a, const Plan& p, cudaStream_t st);
+cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st);
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t st);
+
+// tcgen05 path: whether it supports these dims, its smem need, and the launcher.
+bool tc_supported(const lrkv_dims& d, int* smem_bytes);
+cudaError_t launch_split_tc(const SplitArgs& a, const Plan& p, cudaStream_t st);
+
+int num_sms();
+
+}  // namespace lrkv

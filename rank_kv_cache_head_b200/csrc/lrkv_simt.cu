@@ -1,0 +1,289 @@
+// CUDA-core kernels of liblrkv:
+//  * lrkv_split_simt: split-KV decode attention over a per-head low-rank cache in
+//    fp32 arithmetic, for every dtype combination (the fp32-I/O path, and the
+//    fallback for shapes the tcgen05 kernel does not take);
+//  * lrkv_merge: the log-sum-exp merge of the split partials (Flash Decoding);
+//  * lrkv_append: one new latent row per (batch row, KV head), with the per-token
+//    int8 / e4m3 absmax quantiser.
+// The method: per-head factors W_K,g = A_K,g B_K,g, keys/values rebuilt from the
+// latent as K = Z_K B_K, V = Z_V B_V inside the attention kernel and never written
+// to HBM ("WSVD: Weighted Low-Rank Approximation for Fast and Efficient Execution of
+// Low-Precision Vision-Language Models", sections 2.A and 2.C).
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <math_constants.h>
+
+#include "lrkv_internal.h"
+
+namespace lrkv {
+namespace {
+
+constexpr int kSimtThreads = 256;
+constexpr int kSimtTile = 32;  // tokens per inner tile of the CUDA-core kernel
+
+__device__ __forceinline__ float load_io(const void* p, size_t i, int io_dtype) {
+  if (io_dtype == LRKV_F32) return static_cast<const float*>(p)[i];
+  return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+}
+
+__device__ __forceinline__ float load_lat(const void* p, size_t i, int lat) {
+  switch (lat) {
+    case LRKV_F32: return static_cast<const float*>(p)[i];
+    case LRKV_BF16: return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+    case LRKV_I8: return static_cast<float>(static_cast<const int8_t*>(p)[i]);
+    default: {
+      __nv_fp8_e4m3 v;
+      v.__x = static_cast<const __nv_fp8_storage_t*>(p)[i];
+      return static_cast<float>(v);
+    }
+  }
+}
+
+// Valid length of batch row b under the call's contract; flags violations and
+// treats such a row as empty. Split and merge kernels apply the same rule.
+__device__ __forceinline__ int checked_len(const int32_t* seqlens, int b, int Lcap,
+                                           int max_seqlen, uint32_t* header, bool flag) {
+  int L = seqlens[b];
+  uint32_t bad = 0;
+  if (L < 0 || L > Lcap) bad = LRKV_STATUS_SEQLEN_RANGE;
+  else if (L > max_seqlen) bad = LRKV_STATUS_SEQLEN_HINT;
+  if (bad) {
+    if (flag) atomicOr(header + kStatusWord, bad);
+    return 0;
+  }
+  return L;
+}
+
+// grid (S, Hkv, B); one CTA = one split of one (batch row, KV head), all G query
+// heads of the group. Tiles of 32 tokens: latents -> smem (dequantised), rebuild the
+// K tile = Z_K B_K, scores for the G heads, rebuild the V tile = Z_V B_V, online
+// softmax, accumulate P V. fp32 throughout.
+__global__ void __launch_bounds__(kSimtThreads) lrkv_split_simt(SplitArgs a) {
+  extern __shared__ float sm[];
+  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int d = a.d, r = a.r, G = a.G, T = kSimtTile;
+
+  const int L = checked_len(a.seqlens, b, a.Lcap, a.max_seqlen, a.header, false);
+  const int t_begin = s * a.chunk;
+  const int t_end = min(L, t_begin + a.chunk);
+  if (t_begin >= t_end) return;  // empty split: the merge skips it
+
+  float* bk = sm;                 // [r][d]
+  float* bv = bk + r * d;         // [r][d]
+  float* qs = bv + r * d;         // [G][d]
+  float* zk = qs + G * d;         // [T][r]
+  float* zv = zk + T * r;         // [T][r]
+  float* kv = zv + T * r;         // [T][d+1]
+  float* sc = kv + T * (d + 1);   // [G][T] scores, then probabilities
+  float* acc = sc + G * T;        // [G][d]
+  float* ms = acc + G * d;        // [G] running max (log2 units)
+  float* ls = ms + G;             // [G] running sum
+  float* al = ls + G;             // [G] rescale factor of the current tile
+
+  const size_t fac_base = (size_t)g * r * d;
+  for (int i = tid; i < r * d; i += kSimtThreads) {
+    bk[i] = load_io(a.BK, fac_base + i, a.io_dtype);
+    bv[i] = load_io(a.BV, fac_base + i, a.io_dtype);
+  }
+  const size_t q_base = ((size_t)b * a.Hq + (size_t)g * G) * d;
+  for (int i = tid; i < G * d; i += kSimtThreads) {
+    qs[i] = load_io(a.q, q_base + i, a.io_dtype);
+    acc[i] = 0.f;
+  }
+  if (tid < G) {
+    ms[tid] = -CUDART_INF_F;
+    ls[tid] = 0.f;
+  }
+  const size_t row_base = ((size_t)b * a.Hkv + g) * (size_t)a.Lcap;  // token index base
+  const bool quant = a.latent_dtype == LRKV_I8 || a.latent_dtype == LRKV_E4M3;
+
+  for (int t0 = t_begin; t0 < t_end; t0 += T) {
+    const int n = min(T, t_end - t0);
+    __syncthreads();
+    for (int i = tid; i < T * r; i += kSimtThreads) {
+      const int t = i / r;
+      float vk = 0.f, vv = 0.f;
+      if (t < n) {
+        const size_t tok = row_base + t0 + t;
+        const size_t e = tok * r + (i - t * r);
+        vk = load_lat(a.ZK, e, a.latent_dtype);
+        vv = load_lat(a.ZV, e, a.latent_dtype);
+        if (quant) {
+          vk *= a.SK[tok];
+          vv *= a.SV[tok];
+        }
+      }
+      zk[i] = vk;
+      zv[i] = vv;
+    }
+    __syncthreads();
+    // rebuilt key tile K = Z_K B_K
+    for (int i = tid; i < T * d; i += kSimtThreads) {
+      const int t = i / d, c = i - t * d;
+      float sum = 0.f;
+      for (int k = 0; k < r; ++k) sum = fmaf(zk[t * r + k], bk[k * d + c], sum);
+      kv[t * (d + 1) + c] = sum;
+    }
+    __syncthreads();
+    // scores s[g][t] = q_g . K_t / sqrt(d), in log2 units; masked past the row end
+    for (int pair = warp; pair < G * T; pair += kSimtThreads / 32) {
+      const int gi = pair / T, t = pair - gi * T;
+      float dot = 0.f;
+      for (int c = lane; c < d; c += 32) dot = fmaf(qs[gi * d + c], kv[t * (d + 1) + c], dot);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      if (lane == 0) sc[gi * T + t] = (t < n) ? dot * a.scale_log2 : -CUDART_INF_F;
+    }
+    __syncthreads();
+    // rebuilt value tile V = Z_V B_V (overwrites the key tile)
+    for (int i = tid; i < T * d; i += kSimtThreads) {
+      const int t = i / d, c = i - t * d;
+      float sum = 0.f;
+      for (int k = 0; k < r; ++k) sum = fmaf(zv[t * r + k], bv[k * d + c], sum);
+      kv[t * (d + 1) + c] = sum;
+    }
+    // online softmax, one thread per query head
+    if (tid < G) {
+      const int gi = tid;
+      float mt = -CUDART_INF_F;
+      for (int t = 0; t < n; ++t) mt = fmaxf(mt, sc[gi * T + t]);
+      const float m_old = ms[gi];
+      const float m_new = fmaxf(m_old, mt);
+      const float alpha = exp2f(m_old - m_new);  // 0 on the first tile (m_old = -inf)
+      float sum = 0.f;
+      for (int t = 0; t < T; ++t) {
+        const float p = (t < n) ? exp2f(sc[gi * T + t] - m_new) : 0.f;
+        sc[gi * T + t] = p;
+        sum += p;
+      }
+      ms[gi] = m_new;
+      ls[gi] = ls[gi] * alpha + sum;
+      al[gi] = alpha;
+    }
+    __syncthreads();
+    for (int i = tid; i < G * d; i += kSimtThreads) {
+      const int gi = i / d, c = i - gi * d;
+      float v = acc[i] * al[gi];
+      for (int t = 0; t < n; ++t) v = fmaf(sc[gi * T + t], kv[t * (d + 1) + c], v);
+      acc[i] = v;
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < G * d; i += kSimtThreads) {
+    const int gi = i / d, c = i - gi * d;
+    const size_t h = (size_t)g * G + gi;
+    a.o_part[(((size_t)b * a.Hq + h) * a.S + s) * d + c] = acc[i] / ls[gi];
+  }
+  if (tid < G) {
+    const size_t h = (size_t)g * G + tid;
+    a.lse_part[((size_t)b * a.Hq + h) * a.S + s] = (ms[tid] + log2f(ls[tid])) * CUDART_LN2_F;
+  }
+}
+
+// grid (B * Hq), 128 threads. out[b][h] = sum_s exp(lse_s - LSE) o_s over the
+// non-empty splits of row b; LSE = log sum_s exp(lse_s). Empty row: 0 and -inf.
+__global__ void __launch_bounds__(128) lrkv_merge(MergeArgs a) {
+  const int bh = blockIdx.x;
+  const int b = bh / a.Hq;
+  const int L = checked_len(a.seqlens, b, a.Lcap, a.max_seqlen, a.header,
+                            (bh % a.Hq) == 0 && threadIdx.x == 0);
+  const int ns = min(a.S, (L + a.chunk - 1) / a.chunk);
+  const float* lse = a.lse_part + (size_t)bh * a.S;
+  const float* o = a.o_part + (size_t)bh * a.S * a.d;
+  float mx = -CUDART_INF_F;
+  for (int s = 0; s < ns; ++s) mx = fmaxf(mx, lse[s]);
+  float tot = 0.f;
+  for (int s = 0; s < ns; ++s) tot += expf(lse[s] - mx);
+  const float LSE = (ns > 0) ? mx + logf(tot) : -CUDART_INF_F;
+  for (int c = threadIdx.x; c < a.d; c += blockDim.x) {
+    float v = 0.f;
+    for (int s = 0; s < ns; ++s) v = fmaf(expf(lse[s] - LSE), o[(size_t)s * a.d + c], v);
+    const size_t oi = (size_t)bh * a.d + c;
+    if (a.io_dtype == LRKV_F32) static_cast<float*>(a.out)[oi] = v;
+    else static_cast<__nv_bfloat16*>(a.out)[oi] = __float2bfloat16_rn(v);
+  }
+  if (a.lse_out && threadIdx.x == 0) a.lse_out[bh] = LSE;
+}
+
+// grid (B), 256 threads: one warp per (KV head, K|V) row of batch row b.
+__global__ void __launch_bounds__(256) lrkv_append_kernel(AppendArgs a) {
+  const int b = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int slot = a.seqlens[b];
+  if (slot < 0 || slot >= a.Lcap) {
+    if (threadIdx.x == 0) atomicOr(a.header + kStatusWord, LRKV_STATUS_APPEND_FULL);
+    return;
+  }
+  const int r = a.r;
+  for (int row = warp; row < 2 * a.Hkv; row += blockDim.x / 32) {
+    const int g = row >> 1;
+    const bool is_v = row & 1;
+    const void* src = is_v ? a.zv_new : a.zk_new;
+    void* dst = is_v ? a.ZV : a.ZK;
+    float* sdst = is_v ? a.SV : a.SK;
+    const size_t in_base = ((size_t)b * a.Hkv + g) * r;
+    const size_t tok = ((size_t)b * a.Hkv + g) * (size_t)a.Lcap + slot;
+    const size_t out_base = tok * r;
+    if (a.latent_dtype == LRKV_F32 || a.latent_dtype == LRKV_BF16) {
+      for (int i = lane; i < r; i += 32) {
+        const float z = load_io(src, in_base + i, a.io_dtype);
+        if (a.latent_dtype == LRKV_F32) static_cast<float*>(dst)[out_base + i] = z;
+        else static_cast<__nv_bfloat16*>(dst)[out_base + i] = __float2bfloat16_rn(z);
+      }
+      continue;
+    }
+    float amax = 0.f;
+    for (int i = lane; i < r; i += 32) amax = fmaxf(amax, fabsf(load_io(src, in_base + i, a.io_dtype)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const bool i8 = a.latent_dtype == LRKV_I8;
+    const float scale = (amax == 0.f) ? 1.f : __fdiv_rn(amax, i8 ? 127.f : 448.f);
+    for (int i = lane; i < r; i += 32) {
+      const float v = __fdiv_rn(load_io(src, in_base + i, a.io_dtype), scale);
+      if (i8) {
+        const int c = min(127, max(-127, __float2int_rn(v)));
+        static_cast<int8_t*>(dst)[out_base + i] = static_cast<int8_t>(c);
+      } else {
+        static_cast<__nv_fp8_storage_t*>(dst)[out_base + i] =
+            __nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+      }
+    }
+    if (lane == 0) sdst[tok] = scale;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) a.seqlens[b] = slot + 1;
+}
+
+}  // namespace
+
+size_t simt_smem_bytes(int r, int d, int G) {
+  const int T = kSimtTile;
+  return sizeof(float) * ((size_t)2 * r * d + 2 * (size_t)G * d + 2 * (size_t)T * r +
+                          (size_t)T * (d + 1) + (size_t)G * T + 3 * (size_t)G);
+}
+
+cudaError_t launch_split_simt(const SplitArgs& a, const Plan& p, cudaStream_t st) {
+  static int configured_smem = 0;
+  if (p.smem > configured_smem) {
+    cudaError_t e = cudaFuncSetAttribute(lrkv_split_simt,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
+    if (e != cudaSuccess) return e;
+    configured_smem = p.smem;
+  }
+  dim3 grid(a.S, a.Hkv, a.B);
+  lrkv_split_simt<<<grid, kSimtThreads, p.smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st) {
+  lrkv_merge<<<a.B * a.Hq, 128, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t st) {
+  lrkv_append_kernel<<<a.B, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace lrkv
