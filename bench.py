@@ -65,6 +65,9 @@ def parse():
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--profile", type=int, default=0, metavar="N",
+                    help="no timing: run N eager decode-attention calls on one cache copy "
+                         "and exit (a short, fixed launch sequence for ncu captures)")
     return ap.parse_args()
 
 
@@ -228,6 +231,16 @@ def workload_config(wl, target, plan, algo):
 # ---------------------------------------------------------------------------------------
 
 
+def event_ms(a, b) -> float:
+    """Elapsed ms between two events the library recorded as graph nodes (torch's own
+    elapsed_time only accepts events recorded through torch)."""
+    from cuda.bindings import runtime as rt
+    err, ms = rt.cudaEventElapsedTime(a.cuda_event, b.cuda_event)
+    if int(err) != 0:
+        raise RuntimeError(f"cudaEventElapsedTime failed: {err}")
+    return float(ms)
+
+
 def largest_divisor_at_most(k: int, cap: int) -> int:
     for g in range(min(k, cap), 0, -1):
         if k % g == 0:
@@ -281,6 +294,9 @@ def run_ours(args, rank, world, local):
     G = largest_divisor_at_most(args.steps, 64)
     ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(G)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(G)]
+    for ev in ev_b + ev_e:     # torch creates the underlying CUDA event on first record
+        ev.record(s_main)
+    torch.cuda.synchronize()
 
     def capture(nsteps, timed):
         g = torch.cuda.CUDAGraph()
@@ -336,7 +352,7 @@ def run_ours(args, rank, world, local):
     t1 = time.perf_counter()
     barrier()
     ms = start.elapsed_time(end)
-    split_ms = [ev_b[k].elapsed_time(ev_e[k]) for k in range(G)]  # last replay's launches
+    split_ms = [event_ms(ev_b[k], ev_e[k]) for k in range(G)]  # last replay's launches
     status = lrkv.read_status(ws)
     if status:
         raise RuntimeError(f"device status {status} after the timed region")
@@ -354,6 +370,11 @@ def run_ours(args, rank, world, local):
     for cp in copies:
         cp["seq"].copy_(seq0)
     ke = max(1, args.e2e_steps)
+    # the end-to-end steps keep appending, so their planning hint covers the growth
+    dims_e2e = lrkv.make_dims(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.d_head, wl.rank,
+                              capacity, min(capacity, Lmax + ke // n_copies + 1), wl.io_dtype,
+                              wl.latent_dtype, 0, args.algo)
+    ws_e2e = lrkv.new_workspace(dims_e2e, device=dev)
     uses = [0] * n_copies
     e2e_lat = 0
     for k in range(ke):
@@ -370,17 +391,18 @@ def run_ours(args, rank, world, local):
         es.record()
         for k in range(ke):
             cp = copies[k % n_copies]
-            lrkv.decode_step_host(dims, q_h, zk_h, zv_h, out_h, q_d, zk_d, zv_d, o_d, cp["ZK"],
-                                  cp["ZV"], cp["SK"], cp["SV"], BK, BV, cp["seq"], ws,
-                                  stream=s_main)
+            lrkv.decode_step_host(dims_e2e, q_h, zk_h, zv_h, out_h, q_d, zk_d, zv_d, o_d,
+                                  cp["ZK"], cp["ZV"], cp["SK"], cp["SV"], BK, BV, cp["seq"],
+                                  ws_e2e, stream=s_main)
             s_main.synchronize()          # the step's result is read on the host
             _ = out_h[0, 0, 0].item()
         ee.record()
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(es.elapsed_time(ee), dev)
-    if lrkv.read_status(ws):
-        raise RuntimeError("device status after the end-to-end loop")
+    st_e2e = lrkv.read_status(ws_e2e)
+    if st_e2e:
+        raise RuntimeError(f"device status {st_e2e} after the end-to-end loop")
 
     # ---- numbers -------------------------------------------------------------------------
     peak, peak_kind = peaks()
@@ -431,8 +453,34 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+def run_profile(args):
+    """N eager lrkv_decode_attn calls on one copy of the workload (for profilers)."""
+    wl = WORKLOADS[args.workload]
+    target = seqlens_for(wl)
+    Lmax = int(target.max())
+    capacity = ((Lmax + 7) // 8) * 8
+    inputs = make_inputs(wl, capacity=capacity, seqlens=target)
+    dims = lrkv.make_dims(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.d_head, wl.rank, capacity,
+                          Lmax, wl.io_dtype, wl.latent_dtype, 0, args.algo)
+    dev = {k: (None if v is None else v.cuda()) for k, v in inputs.items()}
+    out = torch.empty_like(dev["q"])
+    ws = lrkv.new_workspace(dims)
+    for _ in range(args.profile):
+        lrkv.decode_attn(dims, dev["q"], dev["ZK"], dev["ZV"], dev["ZK_scale"], dev["ZV_scale"],
+                         dev["BK"], dev["BV"], dev["seqlens"], out, ws)
+    torch.cuda.synchronize()
+    st = lrkv.read_status(ws)
+    print(json.dumps({"profile_calls": args.profile, "workload": wl.name, "status": st,
+                      "plan": lrkv.plan(dims)}))
+    if st:
+        raise SystemExit(1)
+
+
 def main():
     args = parse()
+    if args.profile:
+        run_profile(args)
+        return
     rank, world, local = dist_init()
     try:
         if args.impl == "reference":

@@ -259,6 +259,13 @@ int lrkv_decode_attn_timed(const lrkv_dims* dims, const void* q, const void* ZK,
   a.latent_dtype = dims->latent_dtype;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_head));
 
+  if (p.algo == LRKV_ALGO_TCGEN05 && quant &&
+      ((reinterpret_cast<uintptr_t>(ZK_scale) | reinterpret_cast<uintptr_t>(ZV_scale)) & 15u)) {
+    if (dims->algo == LRKV_ALGO_TCGEN05) return LRKV_ERR_ALIGN;
+    p.algo = LRKV_ALGO_SIMT;
+    p.smem = (int)simt_smem_bytes(dims->rank, dims->d_head, dims->n_q_heads / dims->n_kv_heads);
+    if (p.smem > 227 * 1024) return LRKV_ERR_UNSUPPORTED;
+  }
   record_event(ev_split_begin, st);
   cudaError_t e = (p.algo == LRKV_ALGO_TCGEN05) ? launch_split_tc(a, p, st)
                                                 : launch_split_simt(a, p, st);

@@ -75,7 +75,7 @@ def lib() -> ctypes.CDLL:
         L.lrkv_decode_attn.argtypes = [dp] + [_vp] * 11 + [ctypes.c_size_t, _vp]
         L.lrkv_decode_attn_timed.argtypes = [dp] + [_vp] * 11 + [ctypes.c_size_t, _vp, _vp, _vp]
         L.lrkv_append.argtypes = [dp] + [_vp] * 8 + [ctypes.c_size_t, _vp]
-        L.lrkv_decode_step_host.argtypes = [dp] + [_vp] * 17 + [ctypes.c_size_t, _vp]
+        L.lrkv_decode_step_host.argtypes = [dp] + [_vp] * 16 + [ctypes.c_size_t, _vp]
         L.lrkv_read_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
         _lib = L
     return _lib

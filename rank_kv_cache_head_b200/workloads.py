@@ -137,9 +137,9 @@ def make_inputs(wl: Workload, capacity: Optional[int] = None, poison: Optional[s
 
     io_t = _TORCH_DTYPE[wl.io_dtype]
     out = {
-        "q": torch.from_numpy(q).to(io_t),
-        "BK": torch.from_numpy(BK).to(io_t),
-        "BV": torch.from_numpy(BV).to(io_t),
+        "q": torch.from_numpy(np.ascontiguousarray(q)).to(io_t).contiguous(),
+        "BK": torch.from_numpy(np.ascontiguousarray(BK)).to(io_t).contiguous(),
+        "BV": torch.from_numpy(np.ascontiguousarray(BV)).to(io_t).contiguous(),
         "seqlens": torch.from_numpy(seqlens.copy()),
     }
 
