@@ -67,6 +67,18 @@ constexpr int kSmemLimit = 232448;           // 227 KB opt-in per block
 
 enum LatKind { kLatBF16 = 0, kLatI8 = 1, kLatE4M3 = 2 };
 
+// warpgroups per side: two key-side and two value-side warpgroups alternate tiles for
+// bf16 latents (more independent warps to hide latency); quantised latents keep one
+// of each plus the converter warpgroup (register budget)
+template <int LAT> struct Roles {
+  static constexpr int kNwg = LAT == kLatBF16 ? 2 : 1;
+  static constexpr int kKFirst = 2;                  // warps 0, 1: producer, MMA
+  static constexpr int kVFirst = kKFirst + 4 * kNwg;
+  static constexpr int kDQFirst = kVFirst + 4 * kNwg;
+  static constexpr int kWarps = kDQFirst + (LAT == kLatBF16 ? 0 : 4);
+  static constexpr int kThreads = 32 * kWarps;
+};
+
 struct alignas(64) TcParams {
   CUtensorMap tm_zk, tm_zv, tm_bk, tm_bv, tm_sk, tm_sv;
   SplitArgs a;
@@ -80,15 +92,17 @@ struct alignas(64) TcParams {
   uint32_t off_b;                    // factors: [nbuf] x {BK, BV}, r*256 bytes each
   uint32_t off_q;                    // q of the unit, fp32 [2][16][128]
   uint32_t off_p;                    // P of the tile, fp32 [2][16][128]
+  uint32_t off_x;                    // second value-side warpgroup's output, fp32 [2][16][128]
   uint32_t off_misc;
   uint32_t smem_bytes;
 };
 
 // small shared arrays after the tiles
 struct Misc {
-  float alpha[2][4][16];    // per key-side warp (softmax stream) and head
-  float stat_m[2][4][16];   // unit end: each stream's running max ...
-  float stat_l[2][4][16];   // ... and running sum
+  float alpha[2][4][16];       // per tile slot, key-side warp (softmax stream), head
+  float stat_m[2][2][4][16];   // unit end, per unit parity and warpgroup: each stream's max
+  float stat_l[2][2][4][16];   // ... and running sum
+  float xm[2][16], xl[2][16];  // second value-side warpgroup's merged max and sum
   float scl[2][2][kT];      // per-token scales of the tile (quantised latents)
   int unit[kUR][8];         // b, g, s, t0, t1, ntiles, terminate
   uint32_t tmem_base;
@@ -112,9 +126,11 @@ enum BarIdx {
   BAR_UEMPTY = BAR_UFULL + kUR,       // [kUR] unit descriptor consumed
   BAR_BQFULL = BAR_UEMPTY + kUR,      // [2] factors landed
   BAR_BQEMPTY = BAR_BQFULL + 2,       // [2] factors no longer needed
-  BAR_STFULL = BAR_BQEMPTY + 2,       // [2] unit statistics written
-  BAR_STEMPTY = BAR_STFULL + 2,       // [2] unit statistics read
-  BAR_DQFULL = BAR_STEMPTY + 2,       // [2] bf16 operand tile converted
+  BAR_STFULL = BAR_BQEMPTY + 2,       // [2 x 2] unit statistics written (parity, warpgroup)
+  BAR_STEMPTY = BAR_STFULL + 4,       // [2 x 2] unit statistics read
+  BAR_XFULL = BAR_STEMPTY + 4,        // [2] second value-side warpgroup's result written
+  BAR_XEMPTY = BAR_XFULL + 2,         // [2] ... and read
+  BAR_DQFULL = BAR_XEMPTY + 2,        // [2] bf16 operand tile converted
   BAR_DQEMPTY = BAR_DQFULL + 2,       // [2] bf16 operand tile consumed by MMA2
   BAR_FINAL = BAR_DQEMPTY + 2,
   BAR_COUNT = BAR_FINAL + 1
@@ -156,8 +172,8 @@ __device__ __forceinline__ void raise_timeout(const SplitArgs& a, Misc* ms) {
   if (atomicExch(&ms->status_reported, 1) == 0) atomicOr(a.header + kStatusWord, LRKV_STATUS_TIMEOUT);
 }
 
-template <int LAT, int GP>
-__global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
+template <int LAT, int GP, bool EXACT>
+__global__ void __launch_bounds__(Roles<LAT>::kThreads, 1)
     lrkv_split_tc(const __grid_constant__ TcParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled tiles, by pointer arithmetic on the shared
@@ -168,7 +184,8 @@ __global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
   Misc* ms = reinterpret_cast<Misc*>(smem + p.off_misc);
   const SplitArgs& a = p.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = a.r, G = a.G;
+  const int r = a.r;
+  const int G = EXACT ? GP : a.G;   // heads per KV head; a compile-time constant when exact
   constexpr bool kQuant = LAT != kLatBF16;
   volatile int* abort_flag = &ms->abort_flag;
   auto bar = [&](int i) -> uint32_t { return smem_addr(&ms->bar[i]); };
@@ -188,17 +205,21 @@ __global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
       mbar_init(bar(BAR_VFREE + x), 4);
       mbar_init(bar(BAR_PFULL + x), 4);
       mbar_init(bar(BAR_PFREE + x), 4);
-      mbar_init(bar(BAR_QREADY + x), 4);
+      mbar_init(bar(BAR_QREADY + x), 4 * Roles<LAT>::kNwg);
       mbar_init(bar(BAR_BQFULL + x), 1);
       mbar_init(bar(BAR_BQEMPTY + x), 1);
-      mbar_init(bar(BAR_STFULL + x), 4);
-      mbar_init(bar(BAR_STEMPTY + x), 4);
+      mbar_init(bar(BAR_STFULL + 2 * x), 4);
+      mbar_init(bar(BAR_STFULL + 2 * x + 1), 4);
+      mbar_init(bar(BAR_STEMPTY + 2 * x), 4);
+      mbar_init(bar(BAR_STEMPTY + 2 * x + 1), 4);
+      mbar_init(bar(BAR_XFULL + x), 4);
+      mbar_init(bar(BAR_XEMPTY + x), 4);
       mbar_init(bar(BAR_DQFULL + x), 4);
       mbar_init(bar(BAR_DQEMPTY + x), 1);
     }
     for (int u = 0; u < kUR; ++u) {
       mbar_init(bar(BAR_UFULL + u), 1);
-      mbar_init(bar(BAR_UEMPTY + u), 1 + 4 + 4 + (kQuant ? 4 : 0));
+      mbar_init(bar(BAR_UEMPTY + u), 1 + 8 * Roles<LAT>::kNwg + (kQuant ? 4 : 0));
     }
     mbar_init(bar(BAR_FINAL), 1);
     fence_barrier_init();
@@ -334,6 +355,18 @@ __global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
     const uint32_t id_k = idesc_f16(1, 0, 1, 128, 128);   // Z_K (K-major) x B_K (MN-major)
     const uint32_t id_v = idesc_f16(1, 1, 0, 128, 128);   // B_V^T (MN-major) x Z_V^T (K-major)
     const int ksteps = r / 16;
+    // descriptor pieces fixed for the launch: per K-step byte offsets inside a latent
+    // tile and the constant fields, so each MMA costs a few integer ops to describe
+    uint32_t zoff[8];
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const int byte = ks * 32;
+      zoff[ks] = (uint32_t)((byte / p.W) * (kT * p.W) + (byte % p.W));
+    }
+    const uint64_t zdesc0 = desc_latent(0u, 0, p.W);     // address field zero
+    const uint64_t fdesc0 = desc_factor(0u, 0, r);
+    auto zdesc = [&](uint32_t base, int ks) { return zdesc0 | (uint64_t)(((base + zoff[ks]) >> 4) & 0x3FFFu); };
+    auto fdesc = [&](uint32_t base, int ks) { return fdesc0 | (uint64_t)(((base + 2048u * ks) >> 4) & 0x3FFFu); };
     uint32_t tile_seq = 0;
     int unit_seq = 0;
     bool ok = true;
@@ -352,7 +385,7 @@ __global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
         tc_fence_after();
 #pragma unroll 1
         for (int ks = 0; ks < ksteps; ++ks)
-          mma_ss(tV(x), desc_factor(pend_bv, ks, r), desc_latent(pend_zv, ks, p.W), id_v, ks > 0);
+          mma_ss(tV(x), fdesc(pend_bv, ks), zdesc(pend_zv, ks), id_v, ks > 0);
         tc_commit(bar(BAR_VFULL + x));
         if (!kQuant) tc_commit(bar(BAR_EMPTY + pend_st));
         else tc_commit(bar(BAR_DQEMPTY + x));
@@ -399,7 +432,7 @@ __global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
           tc_fence_after();
 #pragma unroll 1
           for (int ks = 0; ks < ksteps; ++ks)
-            mma_ss(tK(x), desc_latent(szk, ks, p.W), desc_factor(sbk, ks, r), id_k, ks > 0);
+            mma_ss(tK(x), zdesc(szk, ks), fdesc(sbk, ks), id_k, ks > 0);
           tc_commit(bar(BAR_KFULL + x));
         }
         __syncwarp();
@@ -421,18 +454,20 @@ __global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
     __syncwarp();
     int dummy = 0;
     mbar_wait_warp(bar(BAR_FINAL), 0, &dummy, kWaitNs);
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= Roles<LAT>::kKFirst && warp < Roles<LAT>::kVFirst) {
     // ================================ key side ======================================
+    constexpr int kNwg = Roles<LAT>::kNwg;
+    const int wg = (warp - Roles<LAT>::kKFirst) >> 2;   // warpgroup: tiles of this parity
     const int q4 = warp & 3;                 // TMEM lane quarter = softmax stream
     const int row = q4 * 32 + lane;          // token within the tile
     const uint32_t lanebase = (uint32_t)(q4 * 32) << 16;
-    const int tid = threadIdx.x - 128;
+    const int tid = threadIdx.x - 32 * Roles<LAT>::kKFirst;  // across every key-side warp
     float* qs_all = reinterpret_cast<float*>(smem + p.off_q);   // [2][16][128]
     float* ps_all = reinterpret_cast<float*>(smem + p.off_p);   // [2][16][128]
     // chunks of 32 columns loaded per TMEM wait (register budget) and independent
     // partial sums per head (to break the FMA dependency chain)
-    constexpr int kLd = 2;   // 32-column chunks per TMEM wait (register budget)
-    constexpr int kNpk = GP >= 4 ? 1 : 4 / GP;   // partial sums per head
+    constexpr int kLd = GP >= 4 ? 1 : 2;   // 32-column chunks per TMEM wait (register budget)
+    constexpr int kNpk = GP >= 4 ? 1 : 2;   // packed partial sums per head
     uint32_t tile_seq = 0;
     int unit_seq = 0;
     bool ok = true;
@@ -450,7 +485,7 @@ __global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
         float* qw = qs_all + qx * (16 * kD);
         const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q) +
                                   ((size_t)b * a.Hq + (size_t)g * G) * kD;
-        for (int idx = tid; idx < G * (kD / 8); idx += 128) {
+        for (int idx = tid; idx < G * (kD / 8); idx += 128 * kNwg) {
           const int j = idx / (kD / 8), kc = idx % (kD / 8);
           const uint4 raw = *reinterpret_cast<const uint4*>(qg + (size_t)j * kD + kc * 8);
           const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
@@ -473,19 +508,21 @@ __global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
         m_run[j] = -CUDART_INF_F;
         l_run[j] = 0.f;
       }
-      for (int i = 0; i < ntiles && ok; ++i, ++tile_seq) {
-        const int x = (int)(tile_seq & 1u);
-        const uint32_t ph = (tile_seq >> 1) & 1u;
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const uint32_t ts = tile_seq + (uint32_t)i;     // tile index in this CTA's stream
+        if (kNwg == 2 && (int)(ts & 1u) != wg) continue;
+        const int x = (int)(ts & 1u);
+        const uint32_t ph = (ts >> 1) & 1u;
         const int n_valid = min(kT, t1 - (t0 + i * kT));
         if (!mbar_wait_warp(bar(BAR_KFULL + x), ph, abort_flag, kWaitNs)) { ok = false; break; }
         tc_fence_after();
         // scores of this token against the G heads, straight from its fp32 key row;
-        // partial sums per head (by float4 lane of q) keep enough FMAs independent
-        float dot[GP][kNpk];
+        // packed fp32 FMAs, with two partial sums per head when G is small
+        float2 dot[GP][kNpk];
 #pragma unroll
         for (int j = 0; j < GP; ++j)
 #pragma unroll
-          for (int u = 0; u < kNpk; ++u) dot[j][u] = 0.f;
+          for (int u = 0; u < kNpk; ++u) dot[j][u] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c0 = 0; c0 < kD / 32; c0 += kLd) {
           uint32_t v[kLd][32];
@@ -502,14 +539,14 @@ __global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
           for (int e4 = 0; e4 < 8; ++e4) {
 #pragma unroll
             for (int cl = 0; cl < kLd; ++cl) {
+              const float2 k01 = make_float2(__uint_as_float(v[cl][4 * e4 + 0]), __uint_as_float(v[cl][4 * e4 + 1]));
+              const float2 k23 = make_float2(__uint_as_float(v[cl][4 * e4 + 2]), __uint_as_float(v[cl][4 * e4 + 3]));
 #pragma unroll
               for (int j = 0; j < GP; ++j) {
                 if (j < G) {
                   const float4 qq = *reinterpret_cast<const float4*>(qs + j * kD + 32 * (c0 + cl) + 4 * e4);
-                  dot[j][0 % kNpk] = fmaf(__uint_as_float(v[cl][4 * e4 + 0]), qq.x, dot[j][0 % kNpk]);
-                  dot[j][1 % kNpk] = fmaf(__uint_as_float(v[cl][4 * e4 + 1]), qq.y, dot[j][1 % kNpk]);
-                  dot[j][2 % kNpk] = fmaf(__uint_as_float(v[cl][4 * e4 + 2]), qq.z, dot[j][2 % kNpk]);
-                  dot[j][3 % kNpk] = fmaf(__uint_as_float(v[cl][4 * e4 + 3]), qq.w, dot[j][3 % kNpk]);
+                  dot[j][0] = ffma2(k01, make_float2(qq.x, qq.y), dot[j][0]);
+                  dot[j][kNpk - 1] = ffma2(k23, make_float2(qq.z, qq.w), dot[j][kNpk - 1]);
                 }
               }
             }
@@ -523,15 +560,15 @@ __global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
           sv = ms->scl[x][1][row];
         }
         // P(x) and alpha(x) are free once the value side has consumed the tile two back
-        if (tile_seq >= 2 &&
-            !mbar_wait_warp(bar(BAR_PFREE + x), ((tile_seq >> 1) - 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
+        if (ts >= 2 &&
+            !mbar_wait_warp(bar(BAR_PFREE + x), ((ts >> 1) - 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
         float* P = ps_all + x * (16 * kT);
 #pragma unroll
         for (int j = 0; j < GP; ++j) {
           if (j < G) {
             float dj = 0.f;
 #pragma unroll
-            for (int u = 0; u < kNpk; ++u) dj += dot[j][u];
+            for (int u = 0; u < kNpk; ++u) dj += dot[j][u].x + dot[j][u].y;
             const float sj = valid ? dj * sk : -CUDART_INF_F;
             const float m_new = fmaxf(m_run[j], warp_max(sj));   // this stream's running max
             // a stream with no valid token yet keeps max -inf: nothing to rescale
@@ -548,32 +585,35 @@ __global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
         if (lane == 0) mbar_arrive(bar(BAR_PFULL + x));
       }
       if (!ok) break;
-      // unit statistics of this stream for the value side
+      tile_seq += (uint32_t)ntiles;
+      // unit statistics of this warpgroup's streams for the value side
       const int sx = unit_seq & 1;
-      if (unit_seq >= 2 && !mbar_wait_warp(bar(BAR_STEMPTY + sx), ((unit_seq >> 1) - 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
+      if (unit_seq >= 2 && !mbar_wait_warp(bar(BAR_STEMPTY + 2 * sx + wg), ((unit_seq >> 1) - 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
 #pragma unroll
       for (int j = 0; j < GP; ++j) {
         const float lw = warp_sum(l_run[j]);
         if (lane == 0) {
-          ms->stat_l[sx][q4][j] = lw;
-          ms->stat_m[sx][q4][j] = m_run[j];
+          ms->stat_l[sx][wg][q4][j] = lw;
+          ms->stat_m[sx][wg][q4][j] = m_run[j];
         }
       }
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(bar(BAR_STFULL + sx));
+        mbar_arrive(bar(BAR_STFULL + 2 * sx + wg));
         mbar_arrive(bar(BAR_UEMPTY + us));
       }
       ++unit_seq;
     }
     if (!ok) raise_timeout(a, ms);
-  } else if (warp >= 8 && warp < 12) {
+  } else if (warp >= Roles<LAT>::kVFirst && warp < Roles<LAT>::kDQFirst) {
     // ================================ value side ====================================
+    constexpr int kNwg = Roles<LAT>::kNwg;
+    const int wg = (warp - Roles<LAT>::kVFirst) >> 2;   // warpgroup: tiles of this parity
     const int q4 = warp & 3;
     const int c = q4 * 32 + lane;            // output dimension
     const uint32_t lanebase = (uint32_t)(q4 * 32) << 16;
     const float* ps_all = reinterpret_cast<const float*>(smem + p.off_p);
-    constexpr int kLd = (GP <= 2 && !kQuant) ? 4 : 2;   // 32-token chunks per TMEM wait
+    constexpr int kLd = GP >= 4 ? 1 : 2;   // 32-token chunks per TMEM wait (register budget)
     constexpr int kNpv = GP >= 4 ? 1 : 2;               // partial sums per (head, stream)
     uint32_t tile_seq = 0;
     int unit_seq = 0;
@@ -584,17 +624,19 @@ __global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
       const int* d = ms->unit[us];
       if (d[6]) break;
       const int b = d[0], g = d[1], s = d[2], t0 = d[3], t1 = d[4], ntiles = d[5];
-      // per head, softmax stream (token chunk) and partial sum
-      float acc[GP][4][kNpv];
+      // per head and softmax stream (token chunk): packed partial sums
+      float2 acc[GP][4][kNpv];
 #pragma unroll
       for (int j = 0; j < GP; ++j)
 #pragma unroll
         for (int w = 0; w < 4; ++w)
 #pragma unroll
-          for (int u = 0; u < kNpv; ++u) acc[j][w][u] = 0.f;
-      for (int i = 0; i < ntiles && ok; ++i, ++tile_seq) {
-        const int x = (int)(tile_seq & 1u);
-        const uint32_t ph = (tile_seq >> 1) & 1u;
+          for (int u = 0; u < kNpv; ++u) acc[j][w][u] = make_float2(0.f, 0.f);
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const uint32_t ts = tile_seq + (uint32_t)i;
+        if (kNwg == 2 && (int)(ts & 1u) != wg) continue;
+        const int x = (int)(ts & 1u);
+        const uint32_t ph = (ts >> 1) & 1u;
         const int n_valid = min(kT, t1 - (t0 + i * kT));
         if (!mbar_wait_warp(bar(BAR_VFULL + x), ph, abort_flag, kWaitNs)) { ok = false; break; }
         tc_fence_after();
@@ -615,7 +657,10 @@ __global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
                   for (int w = 0; w < 4; ++w) {
                     const float al = ms->alpha[x][w][j];
 #pragma unroll
-                    for (int u = 0; u < kNpv; ++u) acc[j][w][u] *= al;
+                    for (int u = 0; u < kNpv; ++u) {
+                      acc[j][w][u].x *= al;
+                      acc[j][w][u].y *= al;
+                    }
                   }
             }
           }
@@ -645,10 +690,12 @@ __global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
                 if (j < G) {
                   const int w = w0 + wl;
                   const float4 pp = *reinterpret_cast<const float4*>(P + j * kT + 32 * w + 4 * e4);
-                  acc[j][w][0] = fmaf(pp.x, __uint_as_float(v[wl][4 * e4 + 0]), acc[j][w][0]);
-                  acc[j][w][1 % kNpv] = fmaf(pp.y, __uint_as_float(v[wl][4 * e4 + 1]), acc[j][w][1 % kNpv]);
-                  acc[j][w][0] = fmaf(pp.z, __uint_as_float(v[wl][4 * e4 + 2]), acc[j][w][0]);
-                  acc[j][w][1 % kNpv] = fmaf(pp.w, __uint_as_float(v[wl][4 * e4 + 3]), acc[j][w][1 % kNpv]);
+                  acc[j][w][0] = ffma2(make_float2(pp.x, pp.y),
+                                       make_float2(__uint_as_float(v[wl][4 * e4 + 0]), __uint_as_float(v[wl][4 * e4 + 1])),
+                                       acc[j][w][0]);
+                  acc[j][w][kNpv - 1] = ffma2(make_float2(pp.z, pp.w),
+                                              make_float2(__uint_as_float(v[wl][4 * e4 + 2]), __uint_as_float(v[wl][4 * e4 + 3])),
+                                              acc[j][w][kNpv - 1]);
                 }
               }
             }
@@ -659,47 +706,87 @@ __global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
         if (lane == 0) mbar_arrive(bar(BAR_PFREE + x));
       }
       if (!ok) break;
+      tile_seq += (uint32_t)ntiles;
       const int sx = unit_seq & 1;
-      if (!mbar_wait_warp(bar(BAR_STFULL + sx), (unit_seq >> 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
-      // merge the four softmax streams of each head by their log-sum-exp
-      float outv[GP], lse2[GP];
+      if (!mbar_wait_warp(bar(BAR_STFULL + 2 * sx + wg), (unit_seq >> 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
+      // merge this warpgroup's four softmax streams of each head by their log-sum-exp:
+      // numerator num / sum L relative to max M (log2 units)
+      float num[GP], Ms[GP], Ls[GP];
 #pragma unroll
       for (int j = 0; j < GP; ++j) {
-        outv[j] = 0.f;
-        lse2[j] = -CUDART_INF_F;
+        num[j] = 0.f;
+        Ms[j] = -CUDART_INF_F;
+        Ls[j] = 0.f;
         if (j < G) {
-          const float m0 = ms->stat_m[sx][0][j], m1 = ms->stat_m[sx][1][j];
-          const float m2 = ms->stat_m[sx][2][j], m3 = ms->stat_m[sx][3][j];
+          const float m0 = ms->stat_m[sx][wg][0][j], m1 = ms->stat_m[sx][wg][1][j];
+          const float m2 = ms->stat_m[sx][wg][2][j], m3 = ms->stat_m[sx][wg][3][j];
           const float M = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
           // a stream that never saw a valid token (max -inf) contributes nothing
           auto wgt = [&](float m) { return m == -CUDART_INF_F ? 0.f : exp2f(m - M); };
           const float f0 = wgt(m0), f1 = wgt(m1), f2 = wgt(m2), f3 = wgt(m3);
-          const float L = ms->stat_l[sx][0][j] * f0 + ms->stat_l[sx][1][j] * f1 +
-                          ms->stat_l[sx][2][j] * f2 + ms->stat_l[sx][3][j] * f3;
+          Ls[j] = ms->stat_l[sx][wg][0][j] * f0 + ms->stat_l[sx][wg][1][j] * f1 +
+                  ms->stat_l[sx][wg][2][j] * f2 + ms->stat_l[sx][wg][3][j] * f3;
           float aw[4];
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
             aw[w] = 0.f;
 #pragma unroll
-            for (int u = 0; u < kNpv; ++u) aw[w] += acc[j][w][u];
+            for (int u = 0; u < kNpv; ++u) aw[w] += acc[j][w][u].x + acc[j][w][u].y;
           }
-          const float a0 = aw[0], a1 = aw[1], a2 = aw[2], a3 = aw[3];
-          outv[j] = (a0 * f0 + a1 * f1 + a2 * f2 + a3 * f3) / L;
-          lse2[j] = M + log2f(L);
+          num[j] = aw[0] * f0 + aw[1] * f1 + aw[2] * f2 + aw[3] * f3;
+          Ms[j] = M;
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BAR_STEMPTY + sx));
+      if (lane == 0) mbar_arrive(bar(BAR_STEMPTY + 2 * sx + wg));
+      if (kNwg == 2 && wg == 1) {
+        // hand the second warpgroup's merged result to the first
+        float* xo = reinterpret_cast<float*>(smem + p.off_x) + sx * (16 * kD);
+        if (unit_seq >= 2 && !mbar_wait_warp(bar(BAR_XEMPTY + sx), ((unit_seq >> 1) - 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
+#pragma unroll
+        for (int j = 0; j < GP; ++j)
+          if (j < G) {
+            xo[j * kD + c] = num[j];
+            if (c == 0) {
+              ms->xm[sx][j] = Ms[j];
+              ms->xl[sx][j] = Ls[j];
+            }
+          }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bar(BAR_XFULL + sx));
+          mbar_arrive(bar(BAR_UEMPTY + us));
+        }
+        ++unit_seq;
+        continue;
+      }
+      if (kNwg == 2) {
+        const float* xo = reinterpret_cast<const float*>(smem + p.off_x) + sx * (16 * kD);
+        if (!mbar_wait_warp(bar(BAR_XFULL + sx), (unit_seq >> 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
+#pragma unroll
+        for (int j = 0; j < GP; ++j)
+          if (j < G) {
+            const float M1 = ms->xm[sx][j], L1 = ms->xl[sx][j], n1 = xo[j * kD + c];
+            const float M = fmaxf(Ms[j], M1);
+            const float f0 = Ms[j] == -CUDART_INF_F ? 0.f : exp2f(Ms[j] - M);
+            const float f1 = M1 == -CUDART_INF_F ? 0.f : exp2f(M1 - M);
+            num[j] = num[j] * f0 + n1 * f1;
+            Ls[j] = Ls[j] * f0 + L1 * f1;
+            Ms[j] = M;
+          }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_XEMPTY + sx));
+      }
       const size_t hb = (size_t)b * a.Hq + (size_t)g * G;
 #pragma unroll
       for (int j = 0; j < GP; ++j) {
-        if (j < G) a.o_part[((hb + j) * a.S + s) * kD + c] = outv[j];
+        if (j < G) a.o_part[((hb + j) * a.S + s) * kD + c] = num[j] / Ls[j];
       }
       if (c < G) {
         float lc = 0.f;
 #pragma unroll
         for (int j = 0; j < GP; ++j)
-          if (j == c) lc = lse2[j];
+          if (j == c) lc = Ms[j] + log2f(Ls[j]);
         a.lse_part[(hb + c) * a.S + s] = lc * CUDART_LN2_F;
       }
       __syncwarp();
@@ -707,9 +794,9 @@ __global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
       ++unit_seq;
     }
     if (!ok) raise_timeout(a, ms);
-  } else if (kQuant && warp >= 12) {
+  } else if (kQuant && warp >= Roles<LAT>::kDQFirst) {
     // ============================ code -> bf16 converter ============================
-    const int row = (warp - 12) * 32 + lane;   // token within the tile
+    const int row = (warp - Roles<LAT>::kDQFirst) * 32 + lane;   // token within the tile
     const int W = p.W;
     uint32_t tile_seq = 0;
     int unit_seq = 0;
@@ -818,7 +905,7 @@ __global__ void __launch_bounds__(LAT == kLatBF16 ? 384 : 512, 1)
 
 struct Layout {
   int W, nkb, nstage, nbuf;
-  uint32_t off_stage, stage_bytes, off_zop, off_b, off_q, off_p, off_misc, smem;
+  uint32_t off_stage, stage_bytes, off_zop, off_b, off_q, off_p, off_x, off_misc, smem;
 };
 
 bool plan_layout(int r, bool quant, Layout* L) {
@@ -836,6 +923,8 @@ bool plan_layout(int r, bool quant, Layout* L) {
   off += 2u * 16u * 128u * 4u;
   L->off_p = off;
   off += 2u * 16u * 128u * 4u;
+  L->off_x = off;
+  if (!quant) off += 2u * 16u * 128u * 4u;
   L->off_zop = off;
   if (quant) off += 2u * 2u * tile;
   L->off_misc = off;
@@ -851,9 +940,9 @@ bool plan_layout(int r, bool quant, Layout* L) {
   return true;
 }
 
-template <int LAT, int GP>
+template <int LAT, int GP, bool EXACT>
 cudaError_t launch_typed(const TcParams& prm, int grid, cudaStream_t st) {
-  auto kern = lrkv_split_tc<LAT, GP>;
+  auto kern = lrkv_split_tc<LAT, GP, EXACT>;
   static int configured = 0;
   if ((int)prm.smem_bytes > configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -861,18 +950,24 @@ cudaError_t launch_typed(const TcParams& prm, int grid, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured = (int)prm.smem_bytes;
   }
-  kern<<<grid, LAT == kLatBF16 ? 384 : 512, prm.smem_bytes, st>>>(prm);
+  kern<<<grid, Roles<LAT>::kThreads, prm.smem_bytes, st>>>(prm);
   return cudaGetLastError();
 }
 
 template <int LAT>
 cudaError_t launch_g(const TcParams& prm, int grid, cudaStream_t st) {
+  switch (prm.a.G) {
+    case 1: return launch_typed<LAT, 1, true>(prm, grid, st);
+    case 2: return launch_typed<LAT, 2, true>(prm, grid, st);
+    case 4: return launch_typed<LAT, 4, true>(prm, grid, st);
+    case 8: return launch_typed<LAT, 8, true>(prm, grid, st);
+    case 16: return launch_typed<LAT, 16, true>(prm, grid, st);
+    default: break;
+  }
   const int G = prm.a.G;
-  if (G <= 1) return launch_typed<LAT, 1>(prm, grid, st);
-  if (G <= 2) return launch_typed<LAT, 2>(prm, grid, st);
-  if (G <= 4) return launch_typed<LAT, 4>(prm, grid, st);
-  if (G <= 8) return launch_typed<LAT, 8>(prm, grid, st);
-  return launch_typed<LAT, 16>(prm, grid, st);
+  if (G <= 4) return launch_typed<LAT, 4, false>(prm, grid, st);
+  if (G <= 8) return launch_typed<LAT, 8, false>(prm, grid, st);
+  return launch_typed<LAT, 16, false>(prm, grid, st);
 }
 
 }  // namespace
@@ -929,6 +1024,7 @@ cudaError_t launch_split_tc(const SplitArgs& a, const Plan& plan, cudaStream_t s
   prm.off_b = L.off_b;
   prm.off_q = L.off_q;
   prm.off_p = L.off_p;
+  prm.off_x = L.off_x;
   prm.off_misc = L.off_misc;
   prm.smem_bytes = L.smem;
   switch (a.latent_dtype) {
