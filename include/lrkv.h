@@ -198,6 +198,31 @@ int lrkv_decode_step_host(const lrkv_dims* dims, const void* q_host, const void*
                           size_t workspace_bytes, void* stream);
 
 /*
+ * Decode attention for callers that cannot allocate device memory (a host program
+ * without a device memory manager, or a runtime whose memory budget forbids new
+ * allocations while it serves). The paper has no counterpart: this is a deployment
+ * convenience. Same inputs, outputs and semantics as lrkv_decode_attn, but no
+ * workspace argument: the scratch (split partials, status word, scheduler counters)
+ * is a fixed LRKV_NOALLOC_MAX_WORKSPACE_BYTES area inside the library's own device
+ * memory, which every GPU that loads the library holds until the process exits.
+ *  - Allocates nothing. Returns LRKV_ERR_WORKSPACE when lrkv_workspace_bytes(dims)
+ *    exceeds LRKV_NOALLOC_MAX_WORKSPACE_BYTES.
+ *  - The first call on a device looks up the area's device address
+ *    (cudaGetSymbolAddress, once per device, with that device current); make that
+ *    first call before any stream capture.
+ *  - Every call clears the area's header and reuses the rest, which keeps the
+ *    previous call's partials. All calls share one area per device, so calls that can
+ *    overlap on the GPU (different streams without ordering) race: serialise them.
+ *  - status_out (optional, DEVICE pointer): receives this call's device status word
+ *    (LRKV_STATUS_* bits), written on stream after the kernels.
+ */
+#define LRKV_NOALLOC_MAX_WORKSPACE_BYTES (16u << 20)
+int lrkv_decode_attn_noalloc(const lrkv_dims* dims, const void* q, const void* ZK,
+                             const void* ZV, const float* ZK_scale, const float* ZV_scale,
+                             const void* BK, const void* BV, const int32_t* seqlens, void* out,
+                             float* lse_out, uint32_t* status_out, void* stream);
+
+/*
  * Synchronise stream, copy the workspace status word to *status and clear it.
  * Returns 0, or LRKV_ERR_LAUNCH if the copy failed.
  */

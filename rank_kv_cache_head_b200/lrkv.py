@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
         L.lrkv_decode_attn.argtypes = [dp] + [_vp] * 11 + [ctypes.c_size_t, _vp]
         L.lrkv_decode_attn_timed.argtypes = [dp] + [_vp] * 11 + [ctypes.c_size_t, _vp, _vp, _vp]
         L.lrkv_append.argtypes = [dp] + [_vp] * 8 + [ctypes.c_size_t, _vp]
+        L.lrkv_decode_attn_noalloc.argtypes = [dp] + [_vp] * 12
         L.lrkv_decode_step_host.argtypes = [dp] + [_vp] * 16 + [ctypes.c_size_t, _vp]
         L.lrkv_read_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
         _lib = L
@@ -185,6 +186,27 @@ def decode_attn_timed(dims: Dims, q, ZK, ZV, ZK_scale, ZV_scale, BK, BV, seqlens
                                       _stream(stream), *evs)
     if rc:
         raise LrkvError("lrkv_decode_attn_timed", rc)
+
+
+NOALLOC_MAX_WORKSPACE_BYTES = 16 << 20
+
+
+def decode_attn_noalloc(dims: Dims, q, ZK, ZV, ZK_scale, ZV_scale, BK, BV, seqlens, out,
+                        lse_out=None, status_out=None, stream=None) -> None:
+    """lrkv_decode_attn_noalloc: decode attention with the library's fixed scratch area
+    (no workspace argument; for callers that cannot allocate device memory). Calls
+    share one scratch area per device: do not let them overlap on the GPU."""
+    sh = _shapes(dims)
+    args = [
+        _ptr(q, "q", *sh["q"][::-1]), _ptr(ZK, "ZK", *sh["Z"][::-1]), _ptr(ZV, "ZV", *sh["Z"][::-1]),
+        _ptr(ZK_scale, "ZK_scale", *sh["S"][::-1]), _ptr(ZV_scale, "ZV_scale", *sh["S"][::-1]),
+        _ptr(BK, "BK", *sh["B"][::-1]), _ptr(BV, "BV", *sh["B"][::-1]),
+        _ptr(seqlens, "seqlens", *sh["seq"][::-1]), _ptr(out, "out", *sh["q"][::-1]),
+        _ptr(lse_out, "lse_out", *sh["lse"][::-1]),
+        _ptr(status_out, "status_out", (torch.int32,), 1)]
+    rc = lib().lrkv_decode_attn_noalloc(ctypes.byref(dims), *args, _stream(stream))
+    if rc:
+        raise LrkvError("lrkv_decode_attn_noalloc", rc)
 
 
 class PreparedStep:
