@@ -101,14 +101,16 @@ int make_plan(const lrkv_dims* d, Plan* p) {
   int rc = check_dims(d);
   if (rc) return rc;
   const int G = d->n_q_heads / d->n_kv_heads;
-  int tc_smem = 0;
-  const bool tc_ok = tc_supported(*d, &tc_smem);
+  int tc_smem = 0, tc_ctas = 0;
+  const bool tc_ok = tc_supported(*d, &tc_smem, &tc_ctas);
   if (d->algo == LRKV_ALGO_TCGEN05 && !tc_ok) return LRKV_ERR_UNSUPPORTED;
   p->algo = (d->algo == LRKV_ALGO_SIMT || !tc_ok) ? LRKV_ALGO_SIMT : LRKV_ALGO_TCGEN05;
 
   const int tiles_max = std::max(1, (d->max_seqlen + kTile - 1) / kTile);
   const int rows = d->batch * d->n_kv_heads;
-  const int P = num_sms();
+  // persistent CTAs of the split kernel (the tensor-core kernel runs two per SM when
+  // its tiles fit); the SIMT kernel's plan is sized against the SM count
+  const int P = num_sms() * (p->algo == LRKV_ALGO_TCGEN05 ? tc_ctas : 1);
   int chunk_tiles;
   if (d->num_splits > 0) {
     const int S = std::min(d->num_splits, tiles_max);

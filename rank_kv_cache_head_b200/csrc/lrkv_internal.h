@@ -74,8 +74,9 @@ cudaError_t launch_split_simt(const SplitArgs& a, const Plan& p, cudaStream_t st
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t st);
 
-// tcgen05 path: whether it supports these dims, its smem need, and the launcher.
-bool tc_supported(const lrkv_dims& d, int* smem_bytes);
+// tcgen05 path: whether it supports these dims, its shared memory per CTA and CTAs
+// per SM, and the launcher.
+bool tc_supported(const lrkv_dims& d, int* smem_bytes, int* ctas_per_sm);
 cudaError_t launch_split_tc(const SplitArgs& a, const Plan& p, cudaStream_t st);
 
 int num_sms();

@@ -88,15 +88,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
-// Warp-wide form: lane 0 polls the barrier (32 lanes polling one mbarrier cost
-// about ten times more per wait) and the warp-synchronous broadcast of its result
-// orders every lane after lane 0's acquire. The result is the same in all 32 lanes,
-// so a warp never splits around a .sync.aligned tensor-memory instruction.
+// Warp-wide form: every lane waits, then the warp agrees on the result, so a warp
+// never splits around a .sync.aligned tensor-memory instruction. (Polling from all
+// lanes, each with its own acquire, wakes the warp sooner than one lane polling and
+// broadcasting its result.)
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
                                                volatile int* abort_flag, uint64_t limit_ns) {
-  int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, limit_ns) ? 1 : 0;
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+  const bool ok = mbar_wait(bar, parity, abort_flag, limit_ns);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // ---- TMA -----------------------------------------------------------------------------
@@ -128,6 +127,17 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// plain (non-tensor) bulk copy of `bytes` contiguous bytes, global -> shared, completing
+// on an mbarrier; both addresses 16-byte aligned, bytes a multiple of 16
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
@@ -135,6 +145,24 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 // generic-proxy shared-memory writes -> visible to the async proxy (tensor core, TMA)
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---- named barriers ----------------------------------------------------------------------
+
+// Named barrier `id` over `nthreads` threads (whole, converged warps) that also ORs a
+// predicate across them: every participant gets the same answer, so a group of warps
+// can take one decision (carry on, or unwind after a timed-out wait) together.
+__device__ __forceinline__ bool bar_any(uint32_t id, uint32_t nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 // ---- tcgen05: allocation, fences, MMA, commit -------------------------------------------
@@ -234,6 +262,40 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// ---- tcgen05: tensor-memory -> registers, N columns -----------------------------------
+
+// N consecutive 32-bit columns of this thread's lane (32x32b shape). Asynchronous: the
+// registers hold the data only after tmem_wait_ld().
+template <int N> __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t* v);
+template <> __device__ __forceinline__ void tmem_ld_cols<4>(uint32_t taddr, uint32_t* v) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+               : "r"(taddr));
+}
+
+template <> __device__ __forceinline__ void tmem_ld_cols<8>(uint32_t taddr, uint32_t* v) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+               : "r"(taddr));
+}
+
+template <> __device__ __forceinline__ void tmem_ld_cols<16>(uint32_t taddr, uint32_t* v) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+               : "r"(taddr));
+}
+
+template <> __device__ __forceinline__ void tmem_ld_cols<32>(uint32_t taddr, uint32_t* v) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+               : "r"(taddr));
+}
+
+template <> __device__ __forceinline__ void tmem_ld_cols<64>(uint32_t taddr, uint32_t* v) {
+  tmem_ld_cols<32>(taddr, v);
+  tmem_ld_cols<32>(taddr + 32u, v + 32);
+}
+
 // ---- packed fp32 math ----------------------------------------------------------------
 
 // (d.x, d.y) = (a.x * b.x + c.x, a.y * b.y + c.y), one fma.rn.f32x2 instruction
@@ -244,6 +306,26 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
       "fma.rn.f32x2 rc, ra, rb, rc;\n\tmov.b64 {%0, %1}, rc;\n\t}"
       : "=f"(d.x), "=f"(d.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+// packed pairs of fp32 in one 64-bit register: (lo, hi) = (x, y)
+__device__ __forceinline__ uint64_t pack2(float x, float y) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
+  return r;
+}
+
+__device__ __forceinline__ float2 unpack2(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+
+// a * b + c on packed pairs (fma.rn.f32x2)
+__device__ __forceinline__ uint64_t ffma2p(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
 

@@ -10,41 +10,42 @@
 // intermediate written to HBM (same page, section 2.C). Each split writes a
 // normalised partial and its log-sum-exp; lrkv_merge combines the splits.
 //
-// B200 design (one persistent CTA per SM, warp-specialised, mbarrier pipelines):
-//   warp 0      producer: takes (split, b, g) units from an atomic counter, TMA-loads
-//               the unit's factors B_K, B_V once and its latent tiles through a ring
-//               of shared-memory stages;
-//   warp 1      MMA issuer (one thread) and TMEM owner. The rank-r reconstruction,
+// B200 design. Two CTAs share each SM (persistent; 256 tensor-memory columns each),
+// and every CTA is a short warp-specialised pipeline:
+//   warp 0      producer: takes (split, b, g) units from an atomic counter, brings the
+//               unit's factors B_K, B_V and its q rows in once (TMA, bulk copy), and
+//               streams its latent tiles through a ring of shared-memory stages (TMA).
+//   warp 1      MMA issuer and tensor-memory owner. The rank-r reconstruction,
 //               4 r d flops per token, is the dense contraction of the path and runs
 //               on the 5th-generation tensor cores, bf16 x bf16 -> fp32 in TMEM:
 //                 MMA1  Khat   [128 tok x 128 d] = Z_K tile (K-major) x B_K (MN-major)
 //                 MMA2  Vhat^T [128 d x 128 tok] = B_V^T (MN-major) x Z_V tile^T
-//               Keys and values each have a two-slot TMEM ring (128 columns a slot);
-//               MMA2 trails MMA1 by one tile so a key slot is recycled as soon as its
-//               rows have been read.
-//   warps 4-7   key side, one thread per token (TMEM lane): reads its rebuilt key row
-//               (fp32), forms its G scores against q (held in shared memory), and
-//               runs an online softmax. Each of the four warps owns the same 32-token
-//               slice of every tile and keeps its own running max and sum (its own
-//               "stream"), so no cross-warp exchange sits on the per-tile path;
-//               writes P (fp32) and the per-stream rescale factors.
-//   warps 8-11  value side, one thread per output dimension (TMEM lane of Vhat^T):
-//               keeps one accumulator per (head, stream) -- token chunk w of Vhat^T
-//               belongs to stream w -- skips token columns past the row's length
-//               (cache contents beyond seq_len never reach the result), and at the
-//               unit's end merges the four streams by their log-sum-exp and writes
-//               the split partial.
-//   warps 12-15 (int8 / e4m3 latents only) convert each tile's codes to bf16 (exact)
+//               One TMEM slot for each; the next tile's MMA1 starts as soon as the
+//               consumers hold this tile's key rows in registers, and its MMA2 as soon
+//               as they hold the value rows, so the rebuild of tile t+1 runs under the
+//               softmax and P V of tile t.
+//   warps 2-5   one consumer warpgroup. Per tile, each thread first owns a token (a
+//               TMEM lane of Khat): its G scores against q (fp32, in shared memory)
+//               with packed fp32 FMAs; the warpgroup exchanges warp maxima once
+//               (named barrier), updates the running max, and writes P. Then each
+//               thread owns an output dimension (a TMEM lane of Vhat^T) and
+//               accumulates P Vhat over the tile's tokens; token columns past the
+//               row's length are zeroed, so cache contents beyond seq_len never reach
+//               the result. At the unit's end it writes the split partial and LSE.
+//   warp 6      (int8 / e4m3 latents only) converts each tile's codes to bf16 (exact)
 //               for MMA1/2; the per-token scales multiply the scores (K) and are
 //               folded into P (V), which is exact algebra.
+// The scores and P V are matrix-vector work (G <= 16 query rows per KV head) and stay
+// on CUDA cores: as tcgen05 MMAs they would be N = 16 instructions that cost more
+// tensor-pipe time per tile than the tile's HBM time.
 // Every wait is bounded: a role that waits more than a second sets the CTA's abort
-// flag and LRKV_STATUS_TIMEOUT, and all roles unwind, drain their in-flight copies
-// and MMAs, and free TMEM before the CTA exits.
+// flag and LRKV_STATUS_TIMEOUT; the consumer warps take the decision to unwind
+// together at their named barriers; every role drains its in-flight copies and MMAs
+// and TMEM is freed before the CTA exits.
 //
 // Restrictions: io bf16, latents bf16 / int8 / e4m3, d_head = 128, rank a multiple of
 // 16 in [16, 128], G <= 16, max_seq a multiple of 4 for quantised latents.
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <math_constants.h>
 #include <string.h>
@@ -61,23 +62,36 @@ using namespace sm100;
 constexpr int kD = 128;
 constexpr int kT = 128;          // tokens per tile
 constexpr int kUR = 4;           // unit-descriptor ring depth
-constexpr int kMaxStages = 16;
+constexpr int kMaxStages = 8;
 constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s
-constexpr int kSmemLimit = 232448;           // 227 KB opt-in per block
+// dynamic shared memory of one CTA when two share an SM (228 KB per SM, 1 KB of it
+// reserved per CTA), and of a lone CTA (227 KB opt-in)
+constexpr int kSmemPair = 113 * 1024;
+constexpr int kSmemSolo = 227 * 1024;
+constexpr uint32_t kTmemCols = 256;
 
 enum LatKind { kLatBF16 = 0, kLatI8 = 1, kLatE4M3 = 2 };
 
-// warpgroups per side: two key-side and two value-side warpgroups alternate tiles for
-// bf16 latents (more independent warps to hide latency); quantised latents keep one
-// of each plus the converter warpgroup (register budget)
 template <int LAT> struct Roles {
-  static constexpr int kNwg = LAT == kLatBF16 ? 2 : 1;
-  static constexpr int kKFirst = 2;                  // warps 0, 1: producer, MMA
-  static constexpr int kVFirst = kKFirst + 4 * kNwg;
-  static constexpr int kDQFirst = kVFirst + 4 * kNwg;
-  static constexpr int kWarps = kDQFirst + (LAT == kLatBF16 ? 0 : 4);
+  static constexpr int kCons = 2;   // first consumer warp
+  static constexpr int kDQ = 6;     // converter warp (quantised latents)
+  static constexpr int kWarps = LAT == kLatBF16 ? 6 : 7;
   static constexpr int kThreads = 32 * kWarps;
 };
+
+// Consumer batches: kBC TMEM columns are read per tensor-memory wait, together with
+// the q (key phase) or P (value phase) values of the batch for every head, all held in
+// registers so their shared-memory latency overlaps the TMEM read (64 registers of
+// them; 32 under the 128-register budget of the quantised kernel). kCh independent
+// packed accumulators per head keep the FMA chains short.
+template <int LAT, int GP> struct Shape {
+  static constexpr int kQRegs = LAT == kLatBF16 ? 64 : 32;
+  static constexpr int kBC = (kQRegs / GP) < 4 ? 4 : ((kQRegs / GP) > 64 ? 64 : (kQRegs / GP));
+  static constexpr int kCh = GP <= 1 ? 4 : 2;
+};
+
+// named barriers of the consumer warpgroup (id 0 is __syncthreads)
+enum { NB_Q = 1, NB_MAX = 2, NB_P = 3, NB_END = 4 };
 
 struct alignas(64) TcParams {
   CUtensorMap tm_zk, tm_zv, tm_bk, tm_bv, tm_sk, tm_sv;
@@ -86,56 +100,48 @@ struct alignas(64) TcParams {
   int W;        // bytes per swizzled row block of a bf16 latent tile (32/64/128)
   int nkb;      // row blocks per tile (2r / W)
   int nstage;   // TMA ring depth
-  int nbuf;     // factor buffers (1 or 2)
+  int nbuf;     // factor (and q) buffers: 1 or 2
   uint32_t off_stage, stage_bytes;  // TMA ring
-  uint32_t off_zop;                  // bf16 operand ring (quantised latents)
+  uint32_t off_zop;                  // bf16 operand tiles [2][K,V] (quantised latents)
   uint32_t off_b;                    // factors: [nbuf] x {BK, BV}, r*256 bytes each
-  uint32_t off_q;                    // q of the unit, fp32 [2][16][128]
-  uint32_t off_p;                    // P of the tile, fp32 [2][16][128]
-  uint32_t off_x;                    // second value-side warpgroup's output, fp32 [2][16][128]
+  uint32_t off_qraw;                 // q rows of the unit, bf16 [nbuf][G][128]
+  uint32_t off_qs;                   // q of the unit, fp32 scaled [G][128]
+  uint32_t off_p;                    // P of the tile, fp32 [2][G][128]
   uint32_t off_misc;
   uint32_t smem_bytes;
 };
 
-// small shared arrays after the tiles
+// small shared arrays
 struct Misc {
-  float alpha[2][4][16];       // per tile slot, key-side warp (softmax stream), head
-  float stat_m[2][2][4][16];   // unit end, per unit parity and warpgroup: each stream's max
-  float stat_l[2][2][4][16];   // ... and running sum
-  float xm[2][16], xl[2][16];  // second value-side warpgroup's merged max and sum
-  float scl[2][2][kT];      // per-token scales of the tile (quantised latents)
+  float red[2][16][4];      // per tile parity, head, warp: warp maximum of the scores
+  float lsum[16][4];        // unit end: per head, warp: sum of the softmax weights
+  float scl[2][2][kT];      // per tile slot, K/V: per-token scales (quantised latents)
   int unit[kUR][8];         // b, g, s, t0, t1, ntiles, terminate
   uint32_t tmem_base;
   int abort_flag;
   int status_reported;
   int pad;
-  uint64_t bar[96];
+  uint64_t bar[48];
 };
 
 enum BarIdx {
   BAR_FULL = 0,                       // [kMaxStages] TMA tile landed
   BAR_EMPTY = BAR_FULL + kMaxStages,  // [kMaxStages] stage free again
-  BAR_KFULL = BAR_EMPTY + kMaxStages, // [2] key slot rebuilt (MMA1 done)
-  BAR_KFREE = BAR_KFULL + 2,          // [2] key slot read by the key side
-  BAR_VFULL = BAR_KFREE + 2,          // [2] value slot rebuilt (MMA2 done)
-  BAR_VFREE = BAR_VFULL + 2,          // [2] value slot read by the value side
-  BAR_PFULL = BAR_VFREE + 2,          // [2] P and alpha of the tile written
-  BAR_PFREE = BAR_PFULL + 2,          // [2] P and alpha of the tile consumed
-  BAR_QREADY = BAR_PFREE + 2,         // [2] q of the unit in shared memory
-  BAR_UFULL = BAR_QREADY + 2,         // [kUR] unit descriptor written
+  BAR_KFULL = BAR_EMPTY + kMaxStages, // key slot rebuilt (MMA1 done)
+  BAR_KFREE,                          // key slot read into registers
+  BAR_VFULL,                          // value slot rebuilt (MMA2 done)
+  BAR_VFREE,                          // value slot read into registers
+  BAR_UFULL,                          // [kUR] unit descriptor written
   BAR_UEMPTY = BAR_UFULL + kUR,       // [kUR] unit descriptor consumed
-  BAR_BQFULL = BAR_UEMPTY + kUR,      // [2] factors landed
-  BAR_BQEMPTY = BAR_BQFULL + 2,       // [2] factors no longer needed
-  BAR_STFULL = BAR_BQEMPTY + 2,       // [2 x 2] unit statistics written (parity, warpgroup)
-  BAR_STEMPTY = BAR_STFULL + 4,       // [2 x 2] unit statistics read
-  BAR_XFULL = BAR_STEMPTY + 4,        // [2] second value-side warpgroup's result written
-  BAR_XEMPTY = BAR_XFULL + 2,         // [2] ... and read
-  BAR_DQFULL = BAR_XEMPTY + 2,        // [2] bf16 operand tile converted
+  BAR_BQFULL = BAR_UEMPTY + kUR,      // [2] factors and q rows landed
+  BAR_BQEMPTY = BAR_BQFULL + 2,       // [2] factors and q rows no longer needed
+  BAR_DQFULL = BAR_BQEMPTY + 2,       // [2] bf16 operand tile and scales ready
   BAR_DQEMPTY = BAR_DQFULL + 2,       // [2] bf16 operand tile consumed by MMA2
-  BAR_FINAL = BAR_DQEMPTY + 2,
+  BAR_SCFREE = BAR_DQEMPTY + 2,       // [2] scales of the tile read by the consumers
+  BAR_FINAL = BAR_SCFREE + 2,
   BAR_COUNT = BAR_FINAL + 1
 };
-static_assert(BAR_COUNT <= 96, "barrier array too small");
+static_assert(BAR_COUNT <= 48, "barrier array too small");
 
 __device__ __forceinline__ int checked_len_tc(const SplitArgs& a, int b) {
   const int L = a.seqlens[b];
@@ -173,7 +179,7 @@ __device__ __forceinline__ void raise_timeout(const SplitArgs& a, Misc* ms) {
 }
 
 template <int LAT, int GP, bool EXACT>
-__global__ void __launch_bounds__(Roles<LAT>::kThreads, 1)
+__global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
     lrkv_split_tc(const __grid_constant__ TcParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled tiles, by pointer arithmetic on the shared
@@ -196,49 +202,41 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 1)
     ms->status_reported = 0;
     for (int i = 0; i < p.nstage; ++i) {
       mbar_init(bar(BAR_FULL + i), 1);
-      mbar_init(bar(BAR_EMPTY + i), kQuant ? 4 : 1);
+      mbar_init(bar(BAR_EMPTY + i), 1);
     }
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(bar(BAR_KFULL + x), 1);
-      mbar_init(bar(BAR_KFREE + x), 4);
-      mbar_init(bar(BAR_VFULL + x), 1);
-      mbar_init(bar(BAR_VFREE + x), 4);
-      mbar_init(bar(BAR_PFULL + x), 4);
-      mbar_init(bar(BAR_PFREE + x), 4);
-      mbar_init(bar(BAR_QREADY + x), 4 * Roles<LAT>::kNwg);
-      mbar_init(bar(BAR_BQFULL + x), 1);
-      mbar_init(bar(BAR_BQEMPTY + x), 1);
-      mbar_init(bar(BAR_STFULL + 2 * x), 4);
-      mbar_init(bar(BAR_STFULL + 2 * x + 1), 4);
-      mbar_init(bar(BAR_STEMPTY + 2 * x), 4);
-      mbar_init(bar(BAR_STEMPTY + 2 * x + 1), 4);
-      mbar_init(bar(BAR_XFULL + x), 4);
-      mbar_init(bar(BAR_XEMPTY + x), 4);
-      mbar_init(bar(BAR_DQFULL + x), 4);
-      mbar_init(bar(BAR_DQEMPTY + x), 1);
-    }
+    mbar_init(bar(BAR_KFULL), 1);
+    mbar_init(bar(BAR_KFREE), 4);
+    mbar_init(bar(BAR_VFULL), 1);
+    mbar_init(bar(BAR_VFREE), 4);
     for (int u = 0; u < kUR; ++u) {
       mbar_init(bar(BAR_UFULL + u), 1);
-      mbar_init(bar(BAR_UEMPTY + u), 1 + 8 * Roles<LAT>::kNwg + (kQuant ? 4 : 0));
+      mbar_init(bar(BAR_UEMPTY + u), 1 + 4 + (kQuant ? 1 : 0));
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar(BAR_BQFULL + x), 1);
+      mbar_init(bar(BAR_BQEMPTY + x), 2);   // MMA commit + consumers (q read)
+      mbar_init(bar(BAR_DQFULL + x), 1);
+      mbar_init(bar(BAR_DQEMPTY + x), 1);
+      mbar_init(bar(BAR_SCFREE + x), 4);
     }
     mbar_init(bar(BAR_FINAL), 1);
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_addr(&ms->tmem_base), 512);
+    tmem_alloc(smem_addr(&ms->tmem_base), kTmemCols);
     tmem_relinquish();
     tc_fence_before();
   }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ms->tmem_base;
+  const uint32_t tK = tmem;          // Khat: 128 lanes (tokens) x 128 columns (d)
+  const uint32_t tV = tmem + 128u;   // Vhat^T: 128 lanes (d) x 128 columns (tokens)
 
   const uint32_t s_b = sbase + p.off_b;
   const uint32_t fac_bytes = (uint32_t)r * 256u;      // one factor, bf16
   const uint32_t tile_bytes = (uint32_t)kT * 2u * r;  // one bf16 latent tile
-  // TMEM: key slots at columns [0,128) and [128,256), value slots at [256,384), [384,512)
-  auto tK = [&](int x) { return tmem + 128u * x; };
-  auto tV = [&](int x) { return tmem + 256u + 128u * x; };
+  const uint32_t q_bytes = (uint32_t)G * kD * 2u;     // q rows of one unit, bf16
 
   if (warp == 0) {
     // ================================ producer ======================================
@@ -298,11 +296,14 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 1)
       if (leader) {
         const uint32_t sbk = s_b + (uint32_t)bx * 2u * fac_bytes;
         const uint32_t sbv = sbk + fac_bytes;
-        mbar_arrive_expect_tx(bar(BAR_BQFULL + bx), 2u * fac_bytes);
+        mbar_arrive_expect_tx(bar(BAR_BQFULL + bx), 2u * fac_bytes + q_bytes);
         for (int blk = 0; blk < 2; ++blk) {
           tma_load_2d(sbk + (uint32_t)blk * (uint32_t)r * 128u, &p.tm_bk, bar(BAR_BQFULL + bx), blk * 64, g * r);
           tma_load_2d(sbv + (uint32_t)blk * (uint32_t)r * 128u, &p.tm_bv, bar(BAR_BQFULL + bx), blk * 64, g * r);
         }
+        const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q) +
+                                  ((size_t)b * a.Hq + (size_t)g * G) * kD;
+        bulk_load(sbase + p.off_qraw + (uint32_t)bx * q_bytes, qg, q_bytes, bar(BAR_BQFULL + bx));
       }
       last_bq_unit = unit_seq;
       const int row0 = (b * a.Hkv + g) * a.Lcap + t0;
@@ -370,32 +371,6 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 1)
     uint32_t tile_seq = 0;
     int unit_seq = 0;
     bool ok = true;
-    // the tile whose MMA2 is still to be issued (MMA2 trails MMA1 by one tile)
-    bool pend = false;
-    uint32_t pend_seq = 0, pend_zv = 0, pend_bv = 0;
-    int pend_st = 0, pend_bx = 0;
-    bool pend_last = false;
-
-    auto issue_v = [&]() -> bool {
-      const int x = (int)(pend_seq & 1u);
-      if (pend_seq >= 2 &&
-          !mbar_wait_warp(bar(BAR_VFREE + x), ((pend_seq >> 1) - 1) & 1, abort_flag, kWaitNs))
-        return false;
-      if (leader) {
-        tc_fence_after();
-#pragma unroll 1
-        for (int ks = 0; ks < ksteps; ++ks)
-          mma_ss(tV(x), fdesc(pend_bv, ks), zdesc(pend_zv, ks), id_v, ks > 0);
-        tc_commit(bar(BAR_VFULL + x));
-        if (!kQuant) tc_commit(bar(BAR_EMPTY + pend_st));
-        else tc_commit(bar(BAR_DQEMPTY + x));
-        if (pend_last) tc_commit(bar(BAR_BQEMPTY + pend_bx));
-      }
-      __syncwarp();
-      pend = false;
-      return true;
-    };
-
     while (ok) {
       const int us = unit_seq % kUR;
       if (!mbar_wait_warp(bar(BAR_UFULL + us), (unit_seq / kUR) & 1, abort_flag, kWaitNs)) {
@@ -408,7 +383,6 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 1)
       __syncwarp();
       if (leader) mbar_arrive(bar(BAR_UEMPTY + us));
       const int bx = unit_seq % p.nbuf;
-      if (p.nbuf == 1 && pend && !issue_v()) { ok = false; break; }
       if (!mbar_wait_warp(bar(BAR_BQFULL + bx), (unit_seq / p.nbuf) & 1, abort_flag, kWaitNs)) {
         ok = false;
         break;
@@ -427,126 +401,122 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 1)
           if (!mbar_wait_warp(bar(BAR_DQFULL + x), (tile_seq >> 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
           szk = sbase + p.off_zop + (uint32_t)x * 2u * tile_bytes;
         }
-        if (tile_seq >= 2 && !mbar_wait_warp(bar(BAR_KFREE + x), ((tile_seq >> 1) - 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
+        // the key slot is free once the consumers hold the previous tile's key rows
+        if (tile_seq >= 1 && !mbar_wait_warp(bar(BAR_KFREE), (tile_seq - 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
         if (leader) {
           tc_fence_after();
 #pragma unroll 1
           for (int ks = 0; ks < ksteps; ++ks)
-            mma_ss(tK(x), zdesc(szk, ks), fdesc(sbk, ks), id_k, ks > 0);
-          tc_commit(bar(BAR_KFULL + x));
+            mma_ss(tK, zdesc(szk, ks), fdesc(sbk, ks), id_k, ks > 0);
+          tc_commit(bar(BAR_KFULL));
         }
         __syncwarp();
-        if (pend && !issue_v()) { ok = false; break; }
-        pend = true;
-        pend_seq = tile_seq;
-        pend_zv = szk + tile_bytes;
-        pend_bv = sbv;
-        pend_st = st;
-        pend_bx = bx;
-        pend_last = (i == ntiles - 1);
+        if (tile_seq >= 1 && !mbar_wait_warp(bar(BAR_VFREE), (tile_seq - 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
+        if (leader) {
+          tc_fence_after();
+#pragma unroll 1
+          for (int ks = 0; ks < ksteps; ++ks)
+            mma_ss(tV, fdesc(sbv, ks), zdesc(szk + tile_bytes, ks), id_v, ks > 0);
+          tc_commit(bar(BAR_VFULL));
+          if (!kQuant) tc_commit(bar(BAR_EMPTY + st));
+          else tc_commit(bar(BAR_DQEMPTY + x));
+          if (i == ntiles - 1) tc_commit(bar(BAR_BQEMPTY + bx));
+        }
+        __syncwarp();
       }
       ++unit_seq;
     }
-    if (ok && pend) ok = issue_v();
     if (!ok && leader) raise_timeout(a, ms);
     // every MMA issued by this warp completes before TMEM is released
     if (leader) tc_commit(bar(BAR_FINAL));
     __syncwarp();
     int dummy = 0;
     mbar_wait_warp(bar(BAR_FINAL), 0, &dummy, kWaitNs);
-  } else if (warp >= Roles<LAT>::kKFirst && warp < Roles<LAT>::kVFirst) {
-    // ================================ key side ======================================
-    constexpr int kNwg = Roles<LAT>::kNwg;
-    const int wg = (warp - Roles<LAT>::kKFirst) >> 2;   // warpgroup: tiles of this parity
-    const int q4 = warp & 3;                 // TMEM lane quarter = softmax stream
-    const int row = q4 * 32 + lane;          // token within the tile
+  } else if (warp >= Roles<LAT>::kCons && warp < Roles<LAT>::kCons + 4) {
+    // ================================ consumers =====================================
+    constexpr int kBC = Shape<LAT, GP>::kBC;    // TMEM columns per wait
+    constexpr int kCh = Shape<LAT, GP>::kCh;    // packed accumulators per head
+    const int q4 = warp & 3;                    // TMEM lane quarter of this warp
+    const int row = q4 * 32 + lane;             // token of the tile (key phase) and
+    const int c = row;                          // output dimension (value phase)
     const uint32_t lanebase = (uint32_t)(q4 * 32) << 16;
-    const int tid = threadIdx.x - 32 * Roles<LAT>::kKFirst;  // across every key-side warp
-    float* qs_all = reinterpret_cast<float*>(smem + p.off_q);   // [2][16][128]
-    float* ps_all = reinterpret_cast<float*>(smem + p.off_p);   // [2][16][128]
-    // chunks of 32 columns loaded per TMEM wait (register budget) and independent
-    // partial sums per head (to break the FMA dependency chain)
-    constexpr int kLd = GP >= 4 ? 1 : 2;   // 32-column chunks per TMEM wait (register budget)
-    constexpr int kNpk = GP >= 4 ? 1 : 2;   // packed partial sums per head
+    const uint32_t ctid = threadIdx.x - 32 * Roles<LAT>::kCons;
+    float* qs = reinterpret_cast<float*>(smem + p.off_qs);            // [G][128]
+    float* ps_all = reinterpret_cast<float*>(smem + p.off_p);         // [2][G][128]
     uint32_t tile_seq = 0;
     int unit_seq = 0;
-    bool ok = true;
-    while (ok) {
+    bool fail = false;
+    for (;;) {
       const int us = unit_seq % kUR;
-      if (!mbar_wait_warp(bar(BAR_UFULL + us), (unit_seq / kUR) & 1, abort_flag, kWaitNs)) { ok = false; break; }
+      fail = !mbar_wait_warp(bar(BAR_UFULL + us), (unit_seq / kUR) & 1, abort_flag, kWaitNs);
       const int* d = ms->unit[us];
-      if (d[6]) break;
-      const int b = d[0], g = d[1], t0 = d[3], t1 = d[4], ntiles = d[5];
-      // q of the G heads (bf16 in HBM) -> fp32 in shared memory, pre-scaled by
-      // log2(e) / sqrt(d) so the scores come out in log2 units
-      const int qx = unit_seq & 1;
-      const float* qs = qs_all + qx * (16 * kD);
-      {
-        float* qw = qs_all + qx * (16 * kD);
-        const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q) +
-                                  ((size_t)b * a.Hq + (size_t)g * G) * kD;
-        for (int idx = tid; idx < G * (kD / 8); idx += 128 * kNwg) {
-          const int j = idx / (kD / 8), kc = idx % (kD / 8);
-          const uint4 raw = *reinterpret_cast<const uint4*>(qg + (size_t)j * kD + kc * 8);
-          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-          float4 lo, hi;
-          float2 f;
-          f = __bfloat1622float2(h2[0]); lo.x = f.x * a.scale_log2; lo.y = f.y * a.scale_log2;
-          f = __bfloat1622float2(h2[1]); lo.z = f.x * a.scale_log2; lo.w = f.y * a.scale_log2;
-          f = __bfloat1622float2(h2[2]); hi.x = f.x * a.scale_log2; hi.y = f.y * a.scale_log2;
-          f = __bfloat1622float2(h2[3]); hi.z = f.x * a.scale_log2; hi.w = f.y * a.scale_log2;
-          *reinterpret_cast<float4*>(qw + j * kD + kc * 8) = lo;
-          *reinterpret_cast<float4*>(qw + j * kD + kc * 8 + 4) = hi;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BAR_QREADY + qx));
-        if (!mbar_wait_warp(bar(BAR_QREADY + qx), (unit_seq >> 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
+      const bool term = fail ? true : d[6] != 0;
+      const int bx = unit_seq % p.nbuf;
+      if (!term)
+        fail = !mbar_wait_warp(bar(BAR_BQFULL + bx), (unit_seq / p.nbuf) & 1, abort_flag, kWaitNs);
+      if (!term && !fail) {
+        // q of the G heads (bf16, brought in with the factors) -> fp32, pre-scaled by
+        // log2(e) / sqrt(d) so the scores come out in log2 units
+        const __nv_bfloat16* qr = reinterpret_cast<const __nv_bfloat16*>(
+            smem + p.off_qraw + (size_t)bx * (size_t)G * kD * 2u);
+        for (int j = 0; j < G; ++j) qs[j * kD + c] = __bfloat162float(qr[j * kD + c]) * a.scale_log2;
       }
+      if (bar_any(NB_Q, 128, fail)) { fail = true; break; }
+      if (term) break;
+      if (ctid == 0) mbar_arrive(bar(BAR_BQEMPTY + bx));   // q rows read
+      const int b = d[0], g = d[1], s = d[2], t0 = d[3], t1 = d[4], ntiles = d[5];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_UEMPTY + us));
+
       float m_run[GP], l_run[GP];
+      uint64_t acc[GP][kCh];   // packed partial sums of P Vhat, per head
 #pragma unroll
       for (int j = 0; j < GP; ++j) {
         m_run[j] = -CUDART_INF_F;
         l_run[j] = 0.f;
+#pragma unroll
+        for (int u = 0; u < kCh; ++u) acc[j][u] = 0ull;
       }
-      for (int i = 0; i < ntiles && ok; ++i) {
-        const uint32_t ts = tile_seq + (uint32_t)i;     // tile index in this CTA's stream
-        if (kNwg == 2 && (int)(ts & 1u) != wg) continue;
-        const int x = (int)(ts & 1u);
-        const uint32_t ph = (ts >> 1) & 1u;
+      for (int i = 0; i < ntiles; ++i, ++tile_seq) {
+        const uint32_t ph = tile_seq & 1u;           // KFULL / VFULL phase parity
+        const int par = (int)(tile_seq & 1u);        // max / P buffer
         const int n_valid = min(kT, t1 - (t0 + i * kT));
-        if (!mbar_wait_warp(bar(BAR_KFULL + x), ph, abort_flag, kWaitNs)) { ok = false; break; }
-        tc_fence_after();
-        // scores of this token against the G heads, straight from its fp32 key row;
-        // packed fp32 FMAs, with two partial sums per head when G is small
-        float2 dot[GP][kNpk];
+        // ---- key phase: this thread's token, scores against the G heads ----
+        fail = !mbar_wait_warp(bar(BAR_KFULL), ph, abort_flag, kWaitNs);
+        uint64_t dot[GP][kCh];
 #pragma unroll
         for (int j = 0; j < GP; ++j)
 #pragma unroll
-          for (int u = 0; u < kNpk; ++u) dot[j][u] = make_float2(0.f, 0.f);
+          for (int u = 0; u < kCh; ++u) dot[j][u] = 0ull;
+        if (!fail) {
+          tc_fence_after();
 #pragma unroll
-        for (int c0 = 0; c0 < kD / 32; c0 += kLd) {
-          uint32_t v[kLd][32];
+          for (int c0 = 0; c0 < kD; c0 += kBC) {
+            uint32_t v[kBC];
+            tmem_ld_cols<kBC>(tK + lanebase + (uint32_t)c0, v);
+            ulonglong2 qv[GP][kBC / 4];
 #pragma unroll
-          for (int cl = 0; cl < kLd; ++cl) tmem_ld32(tK(x) + lanebase + 32u * (c0 + cl), v[cl]);
-          tmem_wait_ld();
-          if (c0 + kLd == kD / 32) {
-            // every column of the key slot has been read: it can be rebuilt again
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(BAR_KFREE + x));
-          }
+            for (int j = 0; j < GP; ++j)
+              if (j < G)
 #pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {
+                for (int e = 0; e < kBC / 4; ++e)
+                  qv[j][e] = *reinterpret_cast<const ulonglong2*>(qs + j * kD + c0 + 4 * e);
+            tmem_wait_ld();
+            if (c0 + kBC == kD) {
+              // every key column is in registers: the slot can be rebuilt again
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(bar(BAR_KFREE));
+            }
 #pragma unroll
-            for (int cl = 0; cl < kLd; ++cl) {
-              const float2 k01 = make_float2(__uint_as_float(v[cl][4 * e4 + 0]), __uint_as_float(v[cl][4 * e4 + 1]));
-              const float2 k23 = make_float2(__uint_as_float(v[cl][4 * e4 + 2]), __uint_as_float(v[cl][4 * e4 + 3]));
+            for (int e = 0; e < kBC / 4; ++e) {
+              const uint64_t k01 = pack2(__uint_as_float(v[4 * e + 0]), __uint_as_float(v[4 * e + 1]));
+              const uint64_t k23 = pack2(__uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
 #pragma unroll
               for (int j = 0; j < GP; ++j) {
                 if (j < G) {
-                  const float4 qq = *reinterpret_cast<const float4*>(qs + j * kD + 32 * (c0 + cl) + 4 * e4);
-                  dot[j][0] = ffma2(k01, make_float2(qq.x, qq.y), dot[j][0]);
-                  dot[j][kNpk - 1] = ffma2(k23, make_float2(qq.z, qq.w), dot[j][kNpk - 1]);
+                  dot[j][(2 * e) % kCh] = ffma2p(k01, qv[j][e].x, dot[j][(2 * e) % kCh]);
+                  dot[j][(2 * e + 1) % kCh] = ffma2p(k23, qv[j][e].y, dot[j][(2 * e + 1) % kCh]);
                 }
               }
             }
@@ -555,248 +525,137 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 1)
         const bool valid = row < n_valid;
         float sk = 1.f, sv = 1.f;
         if (kQuant) {
-          if (!mbar_wait_warp(bar(BAR_DQFULL + x), ph, abort_flag, kWaitNs)) { ok = false; break; }
-          sk = ms->scl[x][0][row];
-          sv = ms->scl[x][1][row];
+          const int x = (int)(tile_seq & 1u);
+          if (!fail) fail = !mbar_wait_warp(bar(BAR_DQFULL + x), (tile_seq >> 1) & 1, abort_flag, kWaitNs);
+          if (!fail) {
+            sk = ms->scl[x][0][row];
+            sv = ms->scl[x][1][row];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(BAR_SCFREE + x));
+          }
         }
-        // P(x) and alpha(x) are free once the value side has consumed the tile two back
-        if (ts >= 2 &&
-            !mbar_wait_warp(bar(BAR_PFREE + x), ((ts >> 1) - 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
-        float* P = ps_all + x * (16 * kT);
+        float sj[GP];
 #pragma unroll
         for (int j = 0; j < GP; ++j) {
           if (j < G) {
             float dj = 0.f;
 #pragma unroll
-            for (int u = 0; u < kNpk; ++u) dj += dot[j][u].x + dot[j][u].y;
-            const float sj = valid ? dj * sk : -CUDART_INF_F;
-            const float m_new = fmaxf(m_run[j], warp_max(sj));   // this stream's running max
-            // a stream with no valid token yet keeps max -inf: nothing to rescale
-            const float alpha = (m_new == -CUDART_INF_F) ? 1.f : exp2f(m_run[j] - m_new);
-            const float pj = valid ? exp2f(sj - m_new) : 0.f;
-            l_run[j] = l_run[j] * alpha + pj;
+            for (int u = 0; u < kCh; ++u) {
+              const float2 d2 = unpack2(dot[j][u]);
+              dj += d2.x + d2.y;
+            }
+            sj[j] = valid ? dj * sk : -CUDART_INF_F;
+            const float wm = warp_max(sj[j]);
+            if (lane == 0) ms->red[par][j][q4] = wm;
+          }
+        }
+        if (bar_any(NB_MAX, 128, fail)) { fail = true; break; }
+        // ---- online softmax over the tile: one running max per head ----
+        float* P = ps_all + par * (G * kT);
+        float alpha[GP];
+#pragma unroll
+        for (int j = 0; j < GP; ++j) {
+          alpha[j] = 1.f;
+          if (j < G) {
+            const float4 wm = *reinterpret_cast<const float4*>(&ms->red[par][j][0]);
+            const float m_new = fmaxf(m_run[j], fmaxf(fmaxf(wm.x, wm.y), fmaxf(wm.z, wm.w)));
+            alpha[j] = (m_new == -CUDART_INF_F) ? 1.f : exp2f(m_run[j] - m_new);
+            const float pj = valid ? exp2f(sj[j] - m_new) : 0.f;
+            l_run[j] = l_run[j] * alpha[j] + pj;
             m_run[j] = m_new;
             // masked tokens contribute an exact zero (their scale may be anything)
             P[j * kT + row] = valid ? pj * sv : 0.f;
-            if (lane == 0) ms->alpha[x][q4][j] = alpha;
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BAR_PFULL + x));
-      }
-      if (!ok) break;
-      tile_seq += (uint32_t)ntiles;
-      // unit statistics of this warpgroup's streams for the value side
-      const int sx = unit_seq & 1;
-      if (unit_seq >= 2 && !mbar_wait_warp(bar(BAR_STEMPTY + 2 * sx + wg), ((unit_seq >> 1) - 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
-#pragma unroll
-      for (int j = 0; j < GP; ++j) {
-        const float lw = warp_sum(l_run[j]);
-        if (lane == 0) {
-          ms->stat_l[sx][wg][q4][j] = lw;
-          ms->stat_m[sx][wg][q4][j] = m_run[j];
+        // ---- value phase: this thread's output dimension ----
+        fail = !mbar_wait_warp(bar(BAR_VFULL), ph, abort_flag, kWaitNs);
+        uint32_t v[kBC];
+        if (!fail) {
+          tc_fence_after();
+          tmem_ld_cols<kBC>(tV + lanebase, v);   // in flight across the barrier
         }
-      }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar(BAR_STFULL + 2 * sx + wg));
-        mbar_arrive(bar(BAR_UEMPTY + us));
-      }
-      ++unit_seq;
-    }
-    if (!ok) raise_timeout(a, ms);
-  } else if (warp >= Roles<LAT>::kVFirst && warp < Roles<LAT>::kDQFirst) {
-    // ================================ value side ====================================
-    constexpr int kNwg = Roles<LAT>::kNwg;
-    const int wg = (warp - Roles<LAT>::kVFirst) >> 2;   // warpgroup: tiles of this parity
-    const int q4 = warp & 3;
-    const int c = q4 * 32 + lane;            // output dimension
-    const uint32_t lanebase = (uint32_t)(q4 * 32) << 16;
-    const float* ps_all = reinterpret_cast<const float*>(smem + p.off_p);
-    constexpr int kLd = GP >= 4 ? 1 : 2;   // 32-token chunks per TMEM wait (register budget)
-    constexpr int kNpv = GP >= 4 ? 1 : 2;               // partial sums per (head, stream)
-    uint32_t tile_seq = 0;
-    int unit_seq = 0;
-    bool ok = true;
-    while (ok) {
-      const int us = unit_seq % kUR;
-      if (!mbar_wait_warp(bar(BAR_UFULL + us), (unit_seq / kUR) & 1, abort_flag, kWaitNs)) { ok = false; break; }
-      const int* d = ms->unit[us];
-      if (d[6]) break;
-      const int b = d[0], g = d[1], s = d[2], t0 = d[3], t1 = d[4], ntiles = d[5];
-      // per head and softmax stream (token chunk): packed partial sums
-      float2 acc[GP][4][kNpv];
+        const bool stop = bar_any(NB_P, 128, fail);
+        if (stop) {
+          if (!fail) tmem_wait_ld();
+          fail = true;
+          break;
+        }
 #pragma unroll
-      for (int j = 0; j < GP; ++j)
+        for (int j = 0; j < GP; ++j) {
+          if (j < G) {
+            const uint64_t a2 = pack2(alpha[j], alpha[j]);
 #pragma unroll
-        for (int w = 0; w < 4; ++w)
-#pragma unroll
-          for (int u = 0; u < kNpv; ++u) acc[j][w][u] = make_float2(0.f, 0.f);
-      for (int i = 0; i < ntiles && ok; ++i) {
-        const uint32_t ts = tile_seq + (uint32_t)i;
-        if (kNwg == 2 && (int)(ts & 1u) != wg) continue;
-        const int x = (int)(ts & 1u);
-        const uint32_t ph = (ts >> 1) & 1u;
-        const int n_valid = min(kT, t1 - (t0 + i * kT));
-        if (!mbar_wait_warp(bar(BAR_VFULL + x), ph, abort_flag, kWaitNs)) { ok = false; break; }
-        tc_fence_after();
-        const float* P = ps_all + x * (16 * kT);
-#pragma unroll
-        for (int w0 = 0; w0 < 4; w0 += kLd) {
-          uint32_t v[kLd][32];
-#pragma unroll
-          for (int wl = 0; wl < kLd; ++wl) tmem_ld32(tV(x) + lanebase + 32u * (w0 + wl), v[wl]);
-          // the value loads are in flight while P of this tile is awaited
-          if (w0 == 0) {
-            if (!mbar_wait_warp(bar(BAR_PFULL + x), ph, abort_flag, kWaitNs)) ok = false;
-            if (ok) {
-#pragma unroll
-              for (int j = 0; j < GP; ++j)
-                if (j < G)
-#pragma unroll
-                  for (int w = 0; w < 4; ++w) {
-                    const float al = ms->alpha[x][w][j];
-#pragma unroll
-                    for (int u = 0; u < kNpv; ++u) {
-                      acc[j][w][u].x *= al;
-                      acc[j][w][u].y *= al;
-                    }
-                  }
-            }
+            for (int u = 0; u < kCh; ++u) acc[j][u] = ffma2p(acc[j][u], a2, 0ull);
           }
+        }
+#pragma unroll
+        for (int c0 = 0; c0 < kD; c0 += kBC) {
+          if (c0 > 0) tmem_ld_cols<kBC>(tV + lanebase + (uint32_t)c0, v);
+          ulonglong2 pv[GP][kBC / 4];
+#pragma unroll
+          for (int j = 0; j < GP; ++j)
+            if (j < G)
+#pragma unroll
+              for (int e = 0; e < kBC / 4; ++e)
+                pv[j][e] = *reinterpret_cast<const ulonglong2*>(P + j * kT + c0 + 4 * e);
           tmem_wait_ld();
-          if (w0 + kLd == 4) {
+          if (c0 + kBC == kD) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(BAR_VFREE + x));
+            if (lane == 0) mbar_arrive(bar(BAR_VFREE));
           }
-          if (!ok) break;
+          if (n_valid < c0 + kBC) {
+            // token columns past the row's length: exact zeros, whatever the cache holds
 #pragma unroll
-          for (int wl = 0; wl < kLd; ++wl) {
-            const int w = w0 + wl;
-            if (32 * w + 32 > n_valid) {
-              // token columns past the row's length: exact zeros, whatever the cache holds
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (32 * w + e >= n_valid) v[wl][e] = 0u;
-            }
+            for (int e = 0; e < kBC; ++e)
+              if (c0 + e >= n_valid) v[e] = 0u;
           }
 #pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {
+          for (int e = 0; e < kBC / 4; ++e) {
+            const uint64_t v01 = pack2(__uint_as_float(v[4 * e + 0]), __uint_as_float(v[4 * e + 1]));
+            const uint64_t v23 = pack2(__uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
 #pragma unroll
-            for (int wl = 0; wl < kLd; ++wl) {
-#pragma unroll
-              for (int j = 0; j < GP; ++j) {
-                if (j < G) {
-                  const int w = w0 + wl;
-                  const float4 pp = *reinterpret_cast<const float4*>(P + j * kT + 32 * w + 4 * e4);
-                  acc[j][w][0] = ffma2(make_float2(pp.x, pp.y),
-                                       make_float2(__uint_as_float(v[wl][4 * e4 + 0]), __uint_as_float(v[wl][4 * e4 + 1])),
-                                       acc[j][w][0]);
-                  acc[j][w][kNpv - 1] = ffma2(make_float2(pp.z, pp.w),
-                                              make_float2(__uint_as_float(v[wl][4 * e4 + 2]), __uint_as_float(v[wl][4 * e4 + 3])),
-                                              acc[j][w][kNpv - 1]);
-                }
+            for (int j = 0; j < GP; ++j) {
+              if (j < G) {
+                acc[j][(2 * e) % kCh] = ffma2p(pv[j][e].x, v01, acc[j][(2 * e) % kCh]);
+                acc[j][(2 * e + 1) % kCh] = ffma2p(pv[j][e].y, v23, acc[j][(2 * e + 1) % kCh]);
               }
             }
           }
         }
-        if (!ok) break;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BAR_PFREE + x));
       }
-      if (!ok) break;
-      tile_seq += (uint32_t)ntiles;
-      const int sx = unit_seq & 1;
-      if (!mbar_wait_warp(bar(BAR_STFULL + 2 * sx + wg), (unit_seq >> 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
-      // merge this warpgroup's four softmax streams of each head by their log-sum-exp:
-      // numerator num / sum L relative to max M (log2 units)
-      float num[GP], Ms[GP], Ls[GP];
+      if (fail) break;
+      // ---- unit end: the softmax sum over the warpgroup, the partial and its LSE ----
 #pragma unroll
       for (int j = 0; j < GP; ++j) {
-        num[j] = 0.f;
-        Ms[j] = -CUDART_INF_F;
-        Ls[j] = 0.f;
         if (j < G) {
-          const float m0 = ms->stat_m[sx][wg][0][j], m1 = ms->stat_m[sx][wg][1][j];
-          const float m2 = ms->stat_m[sx][wg][2][j], m3 = ms->stat_m[sx][wg][3][j];
-          const float M = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-          // a stream that never saw a valid token (max -inf) contributes nothing
-          auto wgt = [&](float m) { return m == -CUDART_INF_F ? 0.f : exp2f(m - M); };
-          const float f0 = wgt(m0), f1 = wgt(m1), f2 = wgt(m2), f3 = wgt(m3);
-          Ls[j] = ms->stat_l[sx][wg][0][j] * f0 + ms->stat_l[sx][wg][1][j] * f1 +
-                  ms->stat_l[sx][wg][2][j] * f2 + ms->stat_l[sx][wg][3][j] * f3;
-          float aw[4];
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            aw[w] = 0.f;
-#pragma unroll
-            for (int u = 0; u < kNpv; ++u) aw[w] += acc[j][w][u].x + acc[j][w][u].y;
-          }
-          num[j] = aw[0] * f0 + aw[1] * f1 + aw[2] * f2 + aw[3] * f3;
-          Ms[j] = M;
+          const float lw = warp_sum(l_run[j]);
+          if (lane == 0) ms->lsum[j][q4] = lw;
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BAR_STEMPTY + 2 * sx + wg));
-      if (kNwg == 2 && wg == 1) {
-        // hand the second warpgroup's merged result to the first
-        float* xo = reinterpret_cast<float*>(smem + p.off_x) + sx * (16 * kD);
-        if (unit_seq >= 2 && !mbar_wait_warp(bar(BAR_XEMPTY + sx), ((unit_seq >> 1) - 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
-#pragma unroll
-        for (int j = 0; j < GP; ++j)
-          if (j < G) {
-            xo[j * kD + c] = num[j];
-            if (c == 0) {
-              ms->xm[sx][j] = Ms[j];
-              ms->xl[sx][j] = Ls[j];
-            }
-          }
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(bar(BAR_XFULL + sx));
-          mbar_arrive(bar(BAR_UEMPTY + us));
-        }
-        ++unit_seq;
-        continue;
-      }
-      if (kNwg == 2) {
-        const float* xo = reinterpret_cast<const float*>(smem + p.off_x) + sx * (16 * kD);
-        if (!mbar_wait_warp(bar(BAR_XFULL + sx), (unit_seq >> 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
-#pragma unroll
-        for (int j = 0; j < GP; ++j)
-          if (j < G) {
-            const float M1 = ms->xm[sx][j], L1 = ms->xl[sx][j], n1 = xo[j * kD + c];
-            const float M = fmaxf(Ms[j], M1);
-            const float f0 = Ms[j] == -CUDART_INF_F ? 0.f : exp2f(Ms[j] - M);
-            const float f1 = M1 == -CUDART_INF_F ? 0.f : exp2f(M1 - M);
-            num[j] = num[j] * f0 + n1 * f1;
-            Ls[j] = Ls[j] * f0 + L1 * f1;
-            Ms[j] = M;
-          }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BAR_XEMPTY + sx));
-      }
+      bar_any(NB_END, 128, false);
       const size_t hb = (size_t)b * a.Hq + (size_t)g * G;
 #pragma unroll
       for (int j = 0; j < GP; ++j) {
-        if (j < G) a.o_part[((hb + j) * a.S + s) * kD + c] = num[j] / Ls[j];
-      }
-      if (c < G) {
-        float lc = 0.f;
+        if (j < G) {
+          const float4 l4 = *reinterpret_cast<const float4*>(&ms->lsum[j][0]);
+          const float L = (l4.x + l4.y) + (l4.z + l4.w);
+          float num = 0.f;
 #pragma unroll
-        for (int j = 0; j < GP; ++j)
-          if (j == c) lc = Ms[j] + log2f(Ls[j]);
-        a.lse_part[(hb + c) * a.S + s] = lc * CUDART_LN2_F;
+          for (int u = 0; u < kCh; ++u) {
+            const float2 a2 = unpack2(acc[j][u]);
+            num += a2.x + a2.y;
+          }
+          a.o_part[((hb + j) * a.S + s) * kD + c] = num / L;
+          if (c == j) a.lse_part[(hb + j) * a.S + s] = (m_run[j] + log2f(L)) * CUDART_LN2_F;
+        }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BAR_UEMPTY + us));
       ++unit_seq;
     }
-    if (!ok) raise_timeout(a, ms);
-  } else if (kQuant && warp >= Roles<LAT>::kDQFirst) {
+    if (fail) raise_timeout(a, ms);
+  } else if (kQuant && warp >= Roles<LAT>::kDQ) {
     // ============================ code -> bf16 converter ============================
-    const int row = (warp - Roles<LAT>::kDQFirst) * 32 + lane;   // token within the tile
+    // one warp; each thread converts four token rows (lane + 32 k) of the tile
     const int W = p.W;
     uint32_t tile_seq = 0;
     int unit_seq = 0;
@@ -808,6 +667,8 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 1)
       const int* d = ms->unit[us];
       if (d[6]) break;
       const int ntiles = d[5];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_UEMPTY + us));
       for (int i = 0; i < ntiles && ok; ++i, ++tile_seq) {
         const int st = (int)(tile_seq % (uint32_t)p.nstage);
         const int x = (int)(tile_seq & 1u);
@@ -815,56 +676,60 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 1)
         if (tile_seq >= 2) {
           // operand slot x free (MMA2 of the tile two back done) and its scales read
           if (!mbar_wait_warp(bar(BAR_DQEMPTY + x), ((tile_seq >> 1) - 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
-          if (!mbar_wait_warp(bar(BAR_PFULL + x), ((tile_seq >> 1) - 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
+          if (!mbar_wait_warp(bar(BAR_SCFREE + x), ((tile_seq >> 1) - 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
         }
         const uint8_t* stage = smem + p.off_stage + (size_t)st * p.stage_bytes;
         uint8_t* zop = smem + p.off_zop + (size_t)x * 2u * tile_bytes;
+        const float* scs = reinterpret_cast<const float*>(stage + 2 * cb);
 #pragma unroll
-        for (int kv = 0; kv < 2; ++kv) {
-          const uint8_t* src = stage + kv * cb + (size_t)row * r;
-          uint8_t* dst = zop + kv * tile_bytes;
-          for (int k0 = 0; k0 < r; k0 += 16) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(src + k0);
-            const uint8_t* cbytes = reinterpret_cast<const uint8_t*>(&raw);
-            uint32_t w[8];
+        for (int rr = 0; rr < 4; ++rr) {
+          const int row = lane + 32 * rr;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              float f0, f1;
-              if (LAT == kLatI8) {
-                f0 = (float)(int8_t)cbytes[2 * e];
-                f1 = (float)(int8_t)cbytes[2 * e + 1];
-              } else {
-                __nv_fp8_e4m3 c0, c1;
-                c0.__x = cbytes[2 * e];
-                c1.__x = cbytes[2 * e + 1];
-                f0 = (float)c0;
-                f1 = (float)c1;
+          for (int kv = 0; kv < 2; ++kv) {
+            const uint8_t* src = stage + kv * cb + (size_t)row * r;
+            uint8_t* dst = zop + kv * tile_bytes;
+            for (int k0 = 0; k0 < r; k0 += 16) {
+              const uint4 raw = *reinterpret_cast<const uint4*>(src + k0);
+              const uint8_t* cbytes = reinterpret_cast<const uint8_t*>(&raw);
+              uint32_t w[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                float f0, f1;
+                if (LAT == kLatI8) {
+                  f0 = (float)(int8_t)cbytes[2 * e];
+                  f1 = (float)(int8_t)cbytes[2 * e + 1];
+                } else {
+                  __nv_fp8_e4m3 c0, c1;
+                  c0.__x = cbytes[2 * e];
+                  c1.__x = cbytes[2 * e + 1];
+                  f0 = (float)c0;
+                  f1 = (float)c1;
+                }
+                const __nv_bfloat162 bb = __floats2bfloat162_rn(f0, f1);
+                w[e] = *reinterpret_cast<const uint32_t*>(&bb);
               }
-              const __nv_bfloat162 bb = __floats2bfloat162_rn(f0, f1);
-              w[e] = *reinterpret_cast<const uint32_t*>(&bb);
-            }
-            // bf16 bytes [2*k0, 2*k0 + 32) of this row: two 16-byte chunks, swizzled
+              // bf16 bytes [2*k0, 2*k0 + 32) of this row: two 16-byte chunks, swizzled
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              const int byte = 2 * k0 + 16 * half;
-              const int kb = byte / W, inrow = byte % W;
-              const int chunk = inrow >> 4;
-              int sw;
-              if (W == 128) sw = chunk ^ (row & 7);
-              else if (W == 64) sw = chunk ^ ((row >> 1) & 3);
-              else sw = chunk ^ ((row >> 2) & 1);
-              uint4 o;
-              o.x = w[4 * half + 0];
-              o.y = w[4 * half + 1];
-              o.z = w[4 * half + 2];
-              o.w = w[4 * half + 3];
-              *reinterpret_cast<uint4*>(dst + (size_t)kb * (kT * W) + (size_t)row * W + sw * 16) = o;
+              for (int half = 0; half < 2; ++half) {
+                const int byte = 2 * k0 + 16 * half;
+                const int kb = byte / W, inrow = byte % W;
+                const int chunk = inrow >> 4;
+                int sw;
+                if (W == 128) sw = chunk ^ (row & 7);
+                else if (W == 64) sw = chunk ^ ((row >> 1) & 3);
+                else sw = chunk ^ ((row >> 2) & 1);
+                uint4 o;
+                o.x = w[4 * half + 0];
+                o.y = w[4 * half + 1];
+                o.z = w[4 * half + 2];
+                o.w = w[4 * half + 3];
+                *reinterpret_cast<uint4*>(dst + (size_t)kb * (kT * W) + (size_t)row * W + sw * 16) = o;
+              }
             }
           }
+          ms->scl[x][0][row] = scs[row];
+          ms->scl[x][1][row] = scs[kT + row];
         }
-        const float* scs = reinterpret_cast<const float*>(stage + 2 * cb);
-        ms->scl[x][0][row] = scs[row];
-        ms->scl[x][1][row] = scs[kT + row];
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -873,8 +738,6 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 1)
         }
       }
       if (!ok) break;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BAR_UEMPTY + us));
       ++unit_seq;
     }
     if (!ok) raise_timeout(a, ms);
@@ -885,7 +748,7 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, kTmemCols);
   }
   if (threadIdx.x == 0) {
     // the last CTA to finish resets the work counter for the next launch
@@ -904,40 +767,56 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 1)
 // ---------------------------------------------------------------------------------------
 
 struct Layout {
-  int W, nkb, nstage, nbuf;
-  uint32_t off_stage, stage_bytes, off_zop, off_b, off_q, off_p, off_x, off_misc, smem;
+  int W, nkb, nstage, nbuf, ctas_per_sm;
+  uint32_t off_stage, stage_bytes, off_zop, off_b, off_qraw, off_qs, off_p, off_misc, smem;
 };
 
-bool plan_layout(int r, bool quant, Layout* L) {
-  if (r < 16 || r > 128 || r % 16) return false;
+uint32_t round_up(uint32_t x, uint32_t m) { return (x + m - 1) / m * m; }
+
+// Shared-memory layout for `nbuf` factor buffers within `limit` bytes; false when
+// fewer than `min_stages` latent stages fit.
+bool layout_for(int r, int G, bool quant, int nbuf, int limit, int min_stages, Layout* L) {
   const int rowb = 2 * r;
   L->W = (rowb % 128 == 0) ? 128 : (rowb % 64 == 0 ? 64 : 32);
   L->nkb = rowb / L->W;
-  L->nbuf = (r <= 64) ? 2 : 1;
-  const uint32_t tile = 128u * rowb;
-  const uint32_t fac = (uint32_t)r * 256u;
+  L->nbuf = nbuf;
+  const uint32_t tile = 128u * rowb;           // one bf16 latent tile
+  const uint32_t fac = (uint32_t)r * 256u;     // one bf16 factor
   uint32_t off = 0;
-  L->off_b = off;
-  off += L->nbuf * 2u * fac;
-  L->off_q = off;
-  off += 2u * 16u * 128u * 4u;
-  L->off_p = off;
-  off += 2u * 16u * 128u * 4u;
-  L->off_x = off;
-  if (!quant) off += 2u * 16u * 128u * 4u;
+  L->off_b = off;                              // 1024-aligned (128-byte swizzle)
+  off += (uint32_t)nbuf * 2u * fac;
   L->off_zop = off;
   if (quant) off += 2u * 2u * tile;
+  L->off_qraw = off;
+  off += round_up((uint32_t)nbuf * (uint32_t)G * 256u, 128u);
+  L->off_qs = off;
+  off += round_up((uint32_t)G * 512u, 128u);
+  L->off_p = off;
+  off += round_up(2u * (uint32_t)G * 512u, 128u);
   L->off_misc = off;
-  off += (uint32_t)((sizeof(Misc) + 1023) / 1024 * 1024);
+  off = round_up(off + (uint32_t)sizeof(Misc), 1024u);   // swizzled tiles: 1024-aligned
   L->off_stage = off;
-  L->stage_bytes = quant ? (uint32_t)(((2u * 128u * r + 2u * 512u) + 1023u) / 1024u * 1024u) : 2u * tile;
-  const int avail = kSmemLimit - 1024 - (int)off;
+  L->stage_bytes = quant ? round_up(2u * 128u * (uint32_t)r + 2u * 512u, 1024u) : 2u * tile;
+  const int avail = limit - 1024 - (int)off;   // 1024: alignment of the dynamic array
   int ns = avail / (int)L->stage_bytes;
   if (ns > kMaxStages) ns = kMaxStages;
-  if (ns < 2) return false;
+  if (ns < min_stages) return false;
   L->nstage = ns;
   L->smem = 1024u + off + (uint32_t)ns * L->stage_bytes;
   return true;
+}
+
+// Two CTAs per SM when the tiles fit (double-buffered factors when that still leaves
+// three stages), else one CTA with the whole shared memory.
+bool plan_layout(int r, int G, bool quant, Layout* L) {
+  if (r < 16 || r > 128 || r % 16) return false;
+  if (G < 1 || G > 16) return false;
+  L->ctas_per_sm = 2;
+  if (layout_for(r, G, quant, 2, kSmemPair, 3, L)) return true;
+  if (layout_for(r, G, quant, 1, kSmemPair, 2, L)) return true;
+  L->ctas_per_sm = 1;
+  if (layout_for(r, G, quant, 2, kSmemSolo, 3, L)) return true;
+  return layout_for(r, G, quant, 1, kSmemSolo, 2, L);
 }
 
 template <int LAT, int GP, bool EXACT>
@@ -947,6 +826,9 @@ cudaError_t launch_typed(const TcParams& prm, int grid, cudaStream_t st) {
   if ((int)prm.smem_bytes > configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)prm.smem_bytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     configured = (int)prm.smem_bytes;
   }
@@ -972,8 +854,9 @@ cudaError_t launch_g(const TcParams& prm, int grid, cudaStream_t st) {
 
 }  // namespace
 
-bool tc_supported(const lrkv_dims& d, int* smem_bytes) {
+bool tc_supported(const lrkv_dims& d, int* smem_bytes, int* ctas_per_sm) {
   *smem_bytes = 0;
+  *ctas_per_sm = 0;
   if (d.io_dtype != LRKV_BF16 || d.d_head != 128) return false;
   if (d.latent_dtype != LRKV_BF16 && d.latent_dtype != LRKV_I8 && d.latent_dtype != LRKV_E4M3)
     return false;
@@ -983,15 +866,16 @@ bool tc_supported(const lrkv_dims& d, int* smem_bytes) {
   if (quant && d.max_seq % 4 != 0) return false;
   if ((double)d.batch * d.n_kv_heads * d.max_seq >= 2147483647.0) return false;
   Layout L;
-  if (!plan_layout(d.rank, quant, &L)) return false;
+  if (!plan_layout(d.rank, G, quant, &L)) return false;
   *smem_bytes = (int)L.smem;
+  *ctas_per_sm = L.ctas_per_sm;
   return true;
 }
 
 cudaError_t launch_split_tc(const SplitArgs& a, const Plan& plan, cudaStream_t st) {
   const bool quant = a.latent_dtype != LRKV_BF16;
   Layout L;
-  if (!plan_layout(a.r, quant, &L)) return cudaErrorInvalidValue;
+  if (!plan_layout(a.r, a.G, quant, &L)) return cudaErrorInvalidValue;
   TcParams prm;
   memset(&prm, 0, sizeof(prm));
   const uint64_t rows = (uint64_t)a.B * a.Hkv * a.Lcap;
@@ -1022,9 +906,9 @@ cudaError_t launch_split_tc(const SplitArgs& a, const Plan& plan, cudaStream_t s
   prm.stage_bytes = L.stage_bytes;
   prm.off_zop = L.off_zop;
   prm.off_b = L.off_b;
-  prm.off_q = L.off_q;
+  prm.off_qraw = L.off_qraw;
+  prm.off_qs = L.off_qs;
   prm.off_p = L.off_p;
-  prm.off_x = L.off_x;
   prm.off_misc = L.off_misc;
   prm.smem_bytes = L.smem;
   switch (a.latent_dtype) {
