@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "lrkv.h"
 
 namespace lrkv {
@@ -68,6 +70,34 @@ struct AppendArgs {
   int B, Hkv, r, Lcap;
   int io_dtype, latent_dtype;
 };
+
+// Programmatic dependent launch: every kernel of the library is launched so that it
+// may start while the previous kernel of the stream finishes, and waits for that
+// kernel (and so, transitively, every earlier one) before it touches memory they
+// produce; each kernel lets its dependent launch as soon as it has started.
+#ifdef __CUDACC__
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+#endif
+
+// cudaLaunchKernelEx with the programmatic-stream-serialization attribute.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Launchers (return a cudaError_t from the launch).
 cudaError_t launch_split_simt(const SplitArgs& a, const Plan& p, cudaStream_t st);

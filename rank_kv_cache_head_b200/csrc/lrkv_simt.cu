@@ -9,6 +9,8 @@
 // latent as K = Z_K B_K, V = Z_V B_V inside the attention kernel and never written
 // to HBM ("WSVD: Weighted Low-Rank Approximation for Fast and Efficient Execution of
 // Low-Precision Vision-Language Models", sections 2.A and 2.C).
+#include <algorithm>
+
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <math_constants.h>
@@ -60,6 +62,8 @@ __device__ __forceinline__ int checked_len(const int32_t* seqlens, int b, int Lc
 // softmax, accumulate P V. fp32 throughout.
 __global__ void __launch_bounds__(kSimtThreads) lrkv_split_simt(SplitArgs a) {
   extern __shared__ float sm[];
+  griddep_wait();
+  griddep_launch_dependents();
   const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int d = a.d, r = a.r, G = a.G, T = kSimtTile;
@@ -181,66 +185,102 @@ __global__ void __launch_bounds__(kSimtThreads) lrkv_split_simt(SplitArgs a) {
   }
 }
 
-// grid (B * Hq), 128 threads. out[b][h] = sum_s exp(lse_s - LSE) o_s over the
-// non-empty splits of row b; LSE = log sum_s exp(lse_s). Empty row: 0 and -inf.
+// grid (B * Hq), 128 threads (one per output dimension, d <= 128), S floats of dynamic
+// shared memory. out[b][h] = sum_s exp(lse_s - LSE) o_s over the non-empty splits of
+// row b, with LSE = log sum_s exp(lse_s) (the log-sum-exp merge of Flash Decoding); an
+// empty row gives 0 and -inf. The loads that do not depend on the row's length (the
+// first split LSEs and partials) are issued before it is read; warp 0 turns the split
+// LSEs into weights once; every thread sums its dimension with four partial sums.
+// Launched as a programmatic dependent of the split kernel: it waits for the split
+// grid's results before reading them.
 __global__ void __launch_bounds__(128) lrkv_merge(MergeArgs a) {
+  extern __shared__ float wsm[];   // [S] split weights
+  griddep_wait();
+  griddep_launch_dependents();
   const int bh = blockIdx.x;
   const int b = bh / a.Hq;
-  const int L = checked_len(a.seqlens, b, a.Lcap, a.max_seqlen, a.header,
-                            (bh % a.Hq) == 0 && threadIdx.x == 0);
-  const int ns = min(a.S, (L + a.chunk - 1) / a.chunk);
+  const int tid = threadIdx.x, lane = tid & 31;
   const float* lse = a.lse_part + (size_t)bh * a.S;
   const float* o = a.o_part + (size_t)bh * a.S * a.d;
-  float mx = -CUDART_INF_F;
-  for (int s = 0; s < ns; ++s) mx = fmaxf(mx, lse[s]);
-  float tot = 0.f;
-  for (int s = 0; s < ns; ++s) tot += expf(lse[s] - mx);
-  const float LSE = (ns > 0) ? mx + logf(tot) : -CUDART_INF_F;
-  for (int c = threadIdx.x; c < a.d; c += blockDim.x) {
-    float v = 0.f;
-    for (int s = 0; s < ns; ++s) v = fmaf(expf(lse[s] - LSE), o[(size_t)s * a.d + c], v);
-    const size_t oi = (size_t)bh * a.d + c;
-    if (a.io_dtype == LRKV_F32) static_cast<float*>(a.out)[oi] = v;
-    else static_cast<__nv_bfloat16*>(a.out)[oi] = __float2bfloat16_rn(v);
+  constexpr int kPre = 4;
+  const bool active = tid < a.d;
+  float lse0 = -CUDART_INF_F;
+  if (tid < 32 && lane < a.S) lse0 = lse[lane];
+  float opre[kPre];
+#pragma unroll
+  for (int k = 0; k < kPre; ++k) opre[k] = (active && k < a.S) ? o[(size_t)k * a.d + tid] : 0.f;
+  const int L = checked_len(a.seqlens, b, a.Lcap, a.max_seqlen, a.header,
+                            (bh % a.Hq) == 0 && tid == 0);
+  const int ns = min(a.S, (L + a.chunk - 1) / a.chunk);
+  if (tid < 32) {
+    float mx = lane < ns ? lse0 : -CUDART_INF_F;
+    for (int s = lane + 32; s < ns; s += 32) mx = fmaxf(mx, lse[s]);
+#pragma unroll
+    for (int k = 16; k > 0; k >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, k));
+    float tot = lane < ns ? expf(lse0 - mx) : 0.f;
+    for (int s = lane + 32; s < ns; s += 32) tot += expf(lse[s] - mx);
+#pragma unroll
+    for (int k = 16; k > 0; k >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, k);
+    const float LSE = (ns > 0) ? mx + logf(tot) : -CUDART_INF_F;
+    if (lane < ns) wsm[lane] = expf(lse0 - LSE);
+    for (int s = lane + 32; s < ns; s += 32) wsm[s] = expf(lse[s] - LSE);
+    if (a.lse_out && lane == 0) a.lse_out[bh] = LSE;
   }
-  if (a.lse_out && threadIdx.x == 0) a.lse_out[bh] = LSE;
+  __syncthreads();
+  if (!active) return;
+  float v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int k = 0; k < kPre; ++k)
+    if (k < ns) v[k] = wsm[k] * opre[k];
+  int s = kPre;
+  for (; s + 4 <= ns; s += 4) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = fmaf(wsm[s + k], o[(size_t)(s + k) * a.d + tid], v[k]);
+  }
+  for (; s < ns; ++s) v[0] = fmaf(wsm[s], o[(size_t)s * a.d + tid], v[0]);
+  const float r = (v[0] + v[1]) + (v[2] + v[3]);
+  const size_t oi = (size_t)bh * a.d + tid;
+  if (a.io_dtype == LRKV_F32) static_cast<float*>(a.out)[oi] = r;
+  else static_cast<__nv_bfloat16*>(a.out)[oi] = __float2bfloat16_rn(r);
 }
 
-// grid (B), 256 threads: one warp per (KV head, K|V) row of batch row b.
-__global__ void __launch_bounds__(256) lrkv_append_kernel(AppendArgs a) {
-  const int b = blockIdx.x;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int slot = a.seqlens[b];
-  if (slot < 0 || slot >= a.Lcap) {
-    if (threadIdx.x == 0) atomicOr(a.header + kStatusWord, LRKV_STATUS_APPEND_FULL);
+// grid (B), 1024 threads: one warp per (KV head, K|V) row of batch row b, two rows
+// per pass with both rows' loads issued before any store (the kernel is latency-bound).
+// Rows are written at slot seqlens[b]; int8 / e4m3 rows get a per-row absmax scale.
+template <int LAT>
+__device__ __forceinline__ void append_row(const AppendArgs& a, int b, int row, int slot, int lane,
+                                           const float (&z)[8]) {
+  const int r = a.r;
+  const int g = row >> 1;
+  const bool is_v = row & 1;
+  void* dst = is_v ? a.ZV : a.ZK;
+  float* sdst = is_v ? a.SV : a.SK;
+  const size_t tok = ((size_t)b * a.Hkv + g) * (size_t)a.Lcap + slot;
+  const size_t out_base = tok * r;
+  if (LAT == LRKV_F32 || LAT == LRKV_BF16) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i = lane + 32 * k;
+      if (i < r) {
+        if (LAT == LRKV_F32) static_cast<float*>(dst)[out_base + i] = z[k];
+        else static_cast<__nv_bfloat16*>(dst)[out_base + i] = __float2bfloat16_rn(z[k]);
+      }
+    }
     return;
   }
-  const int r = a.r;
-  for (int row = warp; row < 2 * a.Hkv; row += blockDim.x / 32) {
-    const int g = row >> 1;
-    const bool is_v = row & 1;
-    const void* src = is_v ? a.zv_new : a.zk_new;
-    void* dst = is_v ? a.ZV : a.ZK;
-    float* sdst = is_v ? a.SV : a.SK;
-    const size_t in_base = ((size_t)b * a.Hkv + g) * r;
-    const size_t tok = ((size_t)b * a.Hkv + g) * (size_t)a.Lcap + slot;
-    const size_t out_base = tok * r;
-    if (a.latent_dtype == LRKV_F32 || a.latent_dtype == LRKV_BF16) {
-      for (int i = lane; i < r; i += 32) {
-        const float z = load_io(src, in_base + i, a.io_dtype);
-        if (a.latent_dtype == LRKV_F32) static_cast<float*>(dst)[out_base + i] = z;
-        else static_cast<__nv_bfloat16*>(dst)[out_base + i] = __float2bfloat16_rn(z);
-      }
-      continue;
-    }
-    float amax = 0.f;
-    for (int i = lane; i < r; i += 32) amax = fmaxf(amax, fabsf(load_io(src, in_base + i, a.io_dtype)));
+  float amax = 0.f;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const bool i8 = a.latent_dtype == LRKV_I8;
-    const float scale = (amax == 0.f) ? 1.f : __fdiv_rn(amax, i8 ? 127.f : 448.f);
-    for (int i = lane; i < r; i += 32) {
-      const float v = __fdiv_rn(load_io(src, in_base + i, a.io_dtype), scale);
+  for (int k = 0; k < 8; ++k)
+    if (lane + 32 * k < r) amax = fmaxf(amax, fabsf(z[k]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const bool i8 = LAT == LRKV_I8;
+  const float scale = (amax == 0.f) ? 1.f : __fdiv_rn(amax, i8 ? 127.f : 448.f);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int i = lane + 32 * k;
+    if (i < r) {
+      const float v = __fdiv_rn(z[k], scale);
       if (i8) {
         const int c = min(127, max(-127, __float2int_rn(v)));
         static_cast<int8_t*>(dst)[out_base + i] = static_cast<int8_t>(c);
@@ -249,7 +289,42 @@ __global__ void __launch_bounds__(256) lrkv_append_kernel(AppendArgs a) {
             __nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
       }
     }
-    if (lane == 0) sdst[tok] = scale;
+  }
+  if (lane == 0) sdst[tok] = scale;
+}
+
+template <int LAT>
+__global__ void __launch_bounds__(1024) lrkv_append_kernel(AppendArgs a) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int b = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int slot = a.seqlens[b];
+  if (slot < 0 || slot >= a.Lcap) {
+    if (threadIdx.x == 0) atomicOr(a.header + kStatusWord, LRKV_STATUS_APPEND_FULL);
+    return;
+  }
+  const int r = a.r;   // <= 256: at most eight elements a lane
+  const int nrows = 2 * a.Hkv;
+  for (int row0 = warp; row0 < nrows; row0 += 2 * nwarps) {
+    const int row1 = row0 + nwarps;
+    float z0[8], z1[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i = lane + 32 * k;
+      z0[k] = 0.f;
+      z1[k] = 0.f;
+      if (i < r) {
+        const void* s0 = (row0 & 1) ? a.zv_new : a.zk_new;
+        z0[k] = load_io(s0, ((size_t)b * a.Hkv + (row0 >> 1)) * r + i, a.io_dtype);
+        if (row1 < nrows) {
+          const void* s1 = (row1 & 1) ? a.zv_new : a.zk_new;
+          z1[k] = load_io(s1, ((size_t)b * a.Hkv + (row1 >> 1)) * r + i, a.io_dtype);
+        }
+      }
+    }
+    append_row<LAT>(a, b, row0, slot, lane, z0);
+    if (row1 < nrows) append_row<LAT>(a, b, row1, slot, lane, z1);
   }
   __syncthreads();
   if (threadIdx.x == 0) a.seqlens[b] = slot + 1;
@@ -272,18 +347,29 @@ cudaError_t launch_split_simt(const SplitArgs& a, const Plan& p, cudaStream_t st
     configured_smem = p.smem;
   }
   dim3 grid(a.S, a.Hkv, a.B);
-  lrkv_split_simt<<<grid, kSimtThreads, p.smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(lrkv_split_simt, grid, dim3(kSimtThreads), (size_t)p.smem, st, a);
 }
 
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st) {
-  lrkv_merge<<<a.B * a.Hq, 128, 0, st>>>(a);
-  return cudaGetLastError();
+  const size_t smem = (size_t)a.S * sizeof(float);
+  static size_t configured = 48 * 1024;
+  if (smem > configured) {
+    cudaError_t e = cudaFuncSetAttribute(lrkv_merge, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = smem;
+  }
+  return launch_pdl(lrkv_merge, dim3(a.B * a.Hq), dim3(128), smem, st, a);
 }
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t st) {
-  lrkv_append_kernel<<<a.B, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  const int threads = 32 * std::min(32, std::max(1, 2 * a.Hkv));
+  switch (a.latent_dtype) {
+    case LRKV_F32: return launch_pdl(lrkv_append_kernel<LRKV_F32>, dim3(a.B), dim3(threads), 0, st, a);
+    case LRKV_BF16: return launch_pdl(lrkv_append_kernel<LRKV_BF16>, dim3(a.B), dim3(threads), 0, st, a);
+    case LRKV_I8: return launch_pdl(lrkv_append_kernel<LRKV_I8>, dim3(a.B), dim3(threads), 0, st, a);
+    default: return launch_pdl(lrkv_append_kernel<LRKV_E4M3>, dim3(a.B), dim3(threads), 0, st, a);
+  }
 }
 
 }  // namespace lrkv

@@ -126,7 +126,7 @@ struct Misc {
 
 enum BarIdx {
   BAR_FULL = 0,                       // [kMaxStages] TMA tile landed
-  BAR_EMPTY = BAR_FULL + kMaxStages,  // [kMaxStages] stage free again
+  BAR_EMPTY = BAR_FULL + kMaxStages,  // [kMaxStages] stage free again (consumers)
   BAR_KFULL = BAR_EMPTY + kMaxStages, // key slot rebuilt (MMA1 done)
   BAR_KFREE,                          // key slot read into registers
   BAR_VFULL,                          // value slot rebuilt (MMA2 done)
@@ -136,7 +136,7 @@ enum BarIdx {
   BAR_BQFULL = BAR_UEMPTY + kUR,      // [2] factors and q rows landed
   BAR_BQEMPTY = BAR_BQFULL + 2,       // [2] factors and q rows no longer needed
   BAR_DQFULL = BAR_BQEMPTY + 2,       // [2] bf16 operand tile and scales ready
-  BAR_DQEMPTY = BAR_DQFULL + 2,       // [2] bf16 operand tile consumed by MMA2
+  BAR_DQEMPTY = BAR_DQFULL + 2,       // [2] bf16 operand tile consumed (consumers)
   BAR_SCFREE = BAR_DQEMPTY + 2,       // [2] scales of the tile read by the consumers
   BAR_FINAL = BAR_SCFREE + 2,
   BAR_COUNT = BAR_FINAL + 1
@@ -214,12 +214,12 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar(BAR_BQFULL + x), 1);
-      mbar_init(bar(BAR_BQEMPTY + x), 2);   // MMA commit + consumers (q read)
+      mbar_init(bar(BAR_BQEMPTY + x), 1);   // consumers, after the unit's last MMA2
       mbar_init(bar(BAR_DQFULL + x), 1);
       mbar_init(bar(BAR_DQEMPTY + x), 1);
       mbar_init(bar(BAR_SCFREE + x), 4);
     }
-    mbar_init(bar(BAR_FINAL), 1);
+    mbar_init(bar(BAR_FINAL), 3);   // one commit from each MMA-issuing lane
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -227,6 +227,7 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
     tmem_relinquish();
     tc_fence_before();
   }
+  griddep_launch_dependents();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ms->tmem_base;
@@ -252,6 +253,9 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
         prefetch_tmap(&p.tm_sv);
       }
     }
+    // everything this kernel reads from earlier kernels (seqlens, latents, the work
+    // counter) is read here or after units handed out from here
+    griddep_wait();
     const int BH = a.B * a.Hkv;
     uint32_t tile_seq = 0;
     int unit_seq = 0;
@@ -350,8 +354,10 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
     }
   } else if (warp == 1) {
     // ================================ MMA issuer ====================================
-    // The whole warp runs the loop (waits are warp-wide); lane 0 issues the MMAs and
-    // the commits that track them.
+    // The whole warp runs the loop (waits are warp-wide). A commit tracks the MMAs of
+    // the thread that issues it, and one thread's commits complete one after another
+    // (a few hundred cycles each), so the work is spread: lane 0 issues every MMA1 and
+    // its commit; lanes 1 and 2 take the MMA2s of alternate tiles with their commits.
     const bool leader = lane == 0;
     const uint32_t id_k = idesc_f16(1, 0, 1, 128, 128);   // Z_K (K-major) x B_K (MN-major)
     const uint32_t id_v = idesc_f16(1, 1, 0, 128, 128);   // B_V^T (MN-major) x Z_V^T (K-major)
@@ -412,15 +418,12 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
         }
         __syncwarp();
         if (tile_seq >= 1 && !mbar_wait_warp(bar(BAR_VFREE), (tile_seq - 1) & 1, abort_flag, kWaitNs)) { ok = false; break; }
-        if (leader) {
+        if (lane == 1 + (int)(tile_seq & 1u)) {
           tc_fence_after();
 #pragma unroll 1
           for (int ks = 0; ks < ksteps; ++ks)
             mma_ss(tV, fdesc(sbv, ks), zdesc(szk + tile_bytes, ks), id_v, ks > 0);
           tc_commit(bar(BAR_VFULL));
-          if (!kQuant) tc_commit(bar(BAR_EMPTY + st));
-          else tc_commit(bar(BAR_DQEMPTY + x));
-          if (i == ntiles - 1) tc_commit(bar(BAR_BQEMPTY + bx));
         }
         __syncwarp();
       }
@@ -428,7 +431,7 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
     }
     if (!ok && leader) raise_timeout(a, ms);
     // every MMA issued by this warp completes before TMEM is released
-    if (leader) tc_commit(bar(BAR_FINAL));
+    if (lane < 3) tc_commit(bar(BAR_FINAL));
     __syncwarp();
     int dummy = 0;
     mbar_wait_warp(bar(BAR_FINAL), 0, &dummy, kWaitNs);
@@ -463,7 +466,6 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
       }
       if (bar_any(NB_Q, 128, fail)) { fail = true; break; }
       if (term) break;
-      if (ctid == 0) mbar_arrive(bar(BAR_BQEMPTY + bx));   // q rows read
       const int b = d[0], g = d[1], s = d[2], t0 = d[3], t1 = d[4], ntiles = d[5];
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_UEMPTY + us));
@@ -571,6 +573,13 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
         fail = !mbar_wait_warp(bar(BAR_VFULL), ph, abort_flag, kWaitNs);
         uint32_t v[kBC];
         if (!fail) {
+          // MMA1 (KFULL seen) and MMA2 of this tile are complete: their shared-memory
+          // operands are free (a commit would only track its own thread's MMAs)
+          if (ctid == 0) {
+            if (!kQuant) mbar_arrive(bar(BAR_EMPTY + (int)(tile_seq % (uint32_t)p.nstage)));
+            else mbar_arrive(bar(BAR_DQEMPTY + (int)(tile_seq & 1u)));
+            if (i == ntiles - 1) mbar_arrive(bar(BAR_BQEMPTY + bx));   // factors and q rows
+          }
           tc_fence_after();
           tmem_ld_cols<kBC>(tV + lanebase, v);   // in flight across the barrier
         }
@@ -832,8 +841,7 @@ cudaError_t launch_typed(const TcParams& prm, int grid, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured = (int)prm.smem_bytes;
   }
-  kern<<<grid, Roles<LAT>::kThreads, prm.smem_bytes, st>>>(prm);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(Roles<LAT>::kThreads), (size_t)prm.smem_bytes, st, prm);
 }
 
 template <int LAT>
