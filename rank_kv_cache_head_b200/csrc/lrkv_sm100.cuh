@@ -296,6 +296,29 @@ template <> __device__ __forceinline__ void tmem_ld_cols<64>(uint32_t taddr, uin
   tmem_ld_cols<32>(taddr + 32u, v + 32);
 }
 
+// 16 lanes x N repetitions of 8 columns (16x256b shape), 4N registers a thread: with
+// g = lane / 4 and k = lane % 4, registers 4i, 4i+1 hold lane (base + g), columns
+// (8i + 2k, 8i + 2k + 1) and registers 4i+2, 4i+3 the same columns of lane (base + g + 8).
+// Asynchronous like tmem_ld_cols.
+template <int N> __device__ __forceinline__ void tmem_ld16x256(uint32_t taddr, uint32_t* v);
+template <> __device__ __forceinline__ void tmem_ld16x256<2>(uint32_t taddr, uint32_t* v) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+               : "r"(taddr));
+}
+
+template <> __device__ __forceinline__ void tmem_ld16x256<4>(uint32_t taddr, uint32_t* v) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+               : "r"(taddr));
+}
+
+template <> __device__ __forceinline__ void tmem_ld16x256<8>(uint32_t taddr, uint32_t* v) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+               : "r"(taddr));
+}
+
 // ---- packed fp32 math ----------------------------------------------------------------
 
 // (d.x, d.y) = (a.x * b.x + c.x, a.y * b.y + c.y), one fma.rn.f32x2 instruction

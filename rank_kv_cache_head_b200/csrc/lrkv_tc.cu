@@ -79,16 +79,37 @@ template <int LAT> struct Roles {
   static constexpr int kThreads = 32 * kWarps;
 };
 
-// Consumer batches: kBC TMEM columns are read per tensor-memory wait, together with
-// the q (key phase) or P (value phase) values of the batch for every head, all held in
-// registers so their shared-memory latency overlaps the TMEM read (64 registers of
-// them; 32 under the 128-register budget of the quantised kernel). kCh independent
-// packed accumulators per head keep the FMA chains short.
+// Consumer layouts. For G <= 4 each thread reads its slots with the 16x256b shape:
+// four rows of the warp's 32 TMEM lanes (g, g+8, g+16, g+24 with g = lane / 4) and a
+// quarter of the columns (8i + 2k, 8i + 2k + 1 with k = lane % 4). Every q (key phase)
+// or P (value phase) pair a thread loads then serves four rows, and a four-lane
+// reduction completes each row's sum; for G = 1 the thread's q pairs stay in registers
+// for the whole unit. kN repetitions of 8 columns are read per tensor-memory wait.
+// For larger G each thread owns one lane (32x32b shape) and reads kBC columns per wait
+// together with the q or P values of the batch for every head (64 registers of them;
+// 32 under the 128-register budget of the quantised kernel); kCh independent packed
+// accumulators per head keep the FMA chains short.
 template <int LAT, int GP> struct Shape {
+  static constexpr bool kL16 = GP <= 4;
+  static constexpr int kN = LAT == kLatBF16 ? (GP == 1 ? 8 : 4) : (GP == 1 ? 4 : 2);
   static constexpr int kQRegs = LAT == kLatBF16 ? 64 : 32;
   static constexpr int kBC = (kQRegs / GP) < 4 ? 4 : ((kQRegs / GP) > 64 ? 64 : (kQRegs / GP));
   static constexpr int kCh = GP <= 1 ? 4 : 2;
 };
+
+// Sum over the four lanes of a 16x256b row group (lanes 4g .. 4g+3) of four per-row
+// partials a[t] (rows g + 8t); lane 4g + k returns the complete sum of row g + 8k.
+__device__ __forceinline__ float reduce_rows4(float a0, float a1, float a2, float a3, int lane) {
+  const bool b0 = lane & 1, b1 = lane & 2;
+  float keep0 = b0 ? a1 : a0, keep1 = b0 ? a3 : a2;
+  const float send0 = b0 ? a0 : a1, send1 = b0 ? a2 : a3;
+  keep0 += __shfl_xor_sync(0xffffffffu, send0, 1);   // rows b0 and 2 + b0 over lanes k, k^1
+  keep1 += __shfl_xor_sync(0xffffffffu, send1, 1);
+  float keep = b1 ? keep1 : keep0;
+  const float send = b1 ? keep0 : keep1;
+  keep += __shfl_xor_sync(0xffffffffu, send, 2);     // row b0 + 2 b1 over all four lanes
+  return keep;
+}
 
 // named barriers of the consumer warpgroup (id 0 is __syncthreads)
 enum { NB_Q = 1, NB_MAX = 2, NB_P = 3, NB_END = 4 };
@@ -437,12 +458,18 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
     mbar_wait_warp(bar(BAR_FINAL), 0, &dummy, kWaitNs);
   } else if (warp >= Roles<LAT>::kCons && warp < Roles<LAT>::kCons + 4) {
     // ================================ consumers =====================================
-    constexpr int kBC = Shape<LAT, GP>::kBC;    // TMEM columns per wait
-    constexpr int kCh = Shape<LAT, GP>::kCh;    // packed accumulators per head
-    const int q4 = warp & 3;                    // TMEM lane quarter of this warp
-    const int row = q4 * 32 + lane;             // token of the tile (key phase) and
-    const int c = row;                          // output dimension (value phase)
+    constexpr bool kL16 = Shape<LAT, GP>::kL16;  // 16x256b layout (G <= 4)
+    constexpr int kN = Shape<LAT, GP>::kN;       // 16x256b: 8-column repetitions per wait
+    constexpr int kBC = Shape<LAT, GP>::kBC;     // 32x32b: TMEM columns per wait
+    constexpr int kCh = Shape<LAT, GP>::kCh;     // 32x32b: packed accumulators per head
+    const int q4 = warp & 3;                     // TMEM lane quarter of this warp
+    const int g4 = lane >> 2, k4 = lane & 3;     // 16x256b row group and column quarter
+    // the token whose softmax this thread runs (key phase) and the output dimension it
+    // writes (unit end): its own lane (32x32b), or row g + 8k of the quarter (16x256b)
+    const int row = kL16 ? q4 * 32 + g4 + 8 * k4 : q4 * 32 + lane;
+    const int c = row;
     const uint32_t lanebase = (uint32_t)(q4 * 32) << 16;
+    const uint32_t lb1 = (uint32_t)(q4 * 32 + 16) << 16;   // 16x256b: second half of the quarter
     const uint32_t ctid = threadIdx.x - 32 * Roles<LAT>::kCons;
     float* qs = reinterpret_cast<float*>(smem + p.off_qs);            // [G][128]
     float* ps_all = reinterpret_cast<float*>(smem + p.off_p);         // [2][G][128]
@@ -467,60 +494,140 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
       if (bar_any(NB_Q, 128, fail)) { fail = true; break; }
       if (term) break;
       const int b = d[0], g = d[1], s = d[2], t0 = d[3], t1 = d[4], ntiles = d[5];
+      // G = 1, 16x256b: this thread's 16 q pairs (columns 8i + 2k, +1) for the unit
+      uint64_t qreg[(kL16 && GP == 1) ? 16 : 1];
+      if constexpr (kL16 && GP == 1) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) qreg[i] = *reinterpret_cast<const uint64_t*>(qs + 8 * i + 2 * k4);
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_UEMPTY + us));
 
       float m_run[GP], l_run[GP];
-      uint64_t acc[GP][kCh];   // packed partial sums of P Vhat, per head
+      // packed partial sums of P Vhat: per head (32x32b), or per row and head (16x256b)
+      constexpr int kAccA = kL16 ? 4 : GP, kAccB = kL16 ? GP : kCh;
+      uint64_t acc[kAccA][kAccB];
 #pragma unroll
       for (int j = 0; j < GP; ++j) {
         m_run[j] = -CUDART_INF_F;
         l_run[j] = 0.f;
-#pragma unroll
-        for (int u = 0; u < kCh; ++u) acc[j][u] = 0ull;
       }
+#pragma unroll
+      for (int x = 0; x < kAccA; ++x)
+#pragma unroll
+        for (int y = 0; y < kAccB; ++y) acc[x][y] = 0ull;
       for (int i = 0; i < ntiles; ++i, ++tile_seq) {
         const uint32_t ph = tile_seq & 1u;           // KFULL / VFULL phase parity
         const int par = (int)(tile_seq & 1u);        // max / P buffer
         const int n_valid = min(kT, t1 - (t0 + i * kT));
         // ---- key phase: this thread's token, scores against the G heads ----
         fail = !mbar_wait_warp(bar(BAR_KFULL), ph, abort_flag, kWaitNs);
-        uint64_t dot[GP][kCh];
+        float dsum[GP];   // this thread's token: q . Khat for each head
 #pragma unroll
-        for (int j = 0; j < GP; ++j)
+        for (int j = 0; j < GP; ++j) dsum[j] = 0.f;
+        if constexpr (kL16) {
+          uint64_t dot[4][GP];   // rows g, g+8, g+16, g+24 of the quarter
 #pragma unroll
-          for (int u = 0; u < kCh; ++u) dot[j][u] = 0ull;
-        if (!fail) {
-          tc_fence_after();
+          for (int t = 0; t < 4; ++t)
 #pragma unroll
-          for (int c0 = 0; c0 < kD; c0 += kBC) {
-            uint32_t v[kBC];
-            tmem_ld_cols<kBC>(tK + lanebase + (uint32_t)c0, v);
-            ulonglong2 qv[GP][kBC / 4];
+            for (int j = 0; j < GP; ++j) dot[t][j] = 0ull;
+          if (!fail) {
+            tc_fence_after();
 #pragma unroll
-            for (int j = 0; j < GP; ++j)
-              if (j < G)
+            for (int c0 = 0; c0 < kD; c0 += 8 * kN) {
+              uint32_t v0[4 * kN], v1[4 * kN];
+              tmem_ld16x256<kN>(tK + lanebase + (uint32_t)c0, v0);
+              tmem_ld16x256<kN>(tK + lb1 + (uint32_t)c0, v1);
+              uint64_t qp[GP][kN];
 #pragma unroll
-                for (int e = 0; e < kBC / 4; ++e)
-                  qv[j][e] = *reinterpret_cast<const ulonglong2*>(qs + j * kD + c0 + 4 * e);
-            tmem_wait_ld();
-            if (c0 + kBC == kD) {
-              // every key column is in registers: the slot can be rebuilt again
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(bar(BAR_KFREE));
-            }
+              for (int i = 0; i < kN; ++i) {
+                if constexpr (GP == 1) {
+                  qp[0][i] = qreg[c0 / 8 + i];
+                } else {
 #pragma unroll
-            for (int e = 0; e < kBC / 4; ++e) {
-              const uint64_t k01 = pack2(__uint_as_float(v[4 * e + 0]), __uint_as_float(v[4 * e + 1]));
-              const uint64_t k23 = pack2(__uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
-#pragma unroll
-              for (int j = 0; j < GP; ++j) {
-                if (j < G) {
-                  dot[j][(2 * e) % kCh] = ffma2p(k01, qv[j][e].x, dot[j][(2 * e) % kCh]);
-                  dot[j][(2 * e + 1) % kCh] = ffma2p(k23, qv[j][e].y, dot[j][(2 * e + 1) % kCh]);
+                  for (int j = 0; j < GP; ++j)
+                    if (j < G) qp[j][i] = *reinterpret_cast<const uint64_t*>(qs + j * kD + c0 + 8 * i + 2 * k4);
                 }
               }
+              tmem_wait_ld();
+              if (c0 + 8 * kN == kD) {
+                // every key column is in registers: the slot can be rebuilt again
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(BAR_KFREE));
+              }
+#pragma unroll
+              for (int i = 0; i < kN; ++i) {
+                const uint64_t kp[4] = {
+                    pack2(__uint_as_float(v0[4 * i + 0]), __uint_as_float(v0[4 * i + 1])),
+                    pack2(__uint_as_float(v0[4 * i + 2]), __uint_as_float(v0[4 * i + 3])),
+                    pack2(__uint_as_float(v1[4 * i + 0]), __uint_as_float(v1[4 * i + 1])),
+                    pack2(__uint_as_float(v1[4 * i + 2]), __uint_as_float(v1[4 * i + 3]))};
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+#pragma unroll
+                  for (int j = 0; j < GP; ++j)
+                    if (j < G) dot[t][j] = ffma2p(kp[t], qp[j][i], dot[t][j]);
+              }
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < GP; ++j) {
+            if (j < G) {
+              float a4[4];
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                const float2 d2 = unpack2(dot[t][j]);
+                a4[t] = d2.x + d2.y;
+              }
+              dsum[j] = reduce_rows4(a4[0], a4[1], a4[2], a4[3], lane);
+            }
+          }
+        } else {
+          uint64_t dot[GP][kCh];
+#pragma unroll
+          for (int j = 0; j < GP; ++j)
+#pragma unroll
+            for (int u = 0; u < kCh; ++u) dot[j][u] = 0ull;
+          if (!fail) {
+            tc_fence_after();
+#pragma unroll
+            for (int c0 = 0; c0 < kD; c0 += kBC) {
+              uint32_t v[kBC];
+              tmem_ld_cols<kBC>(tK + lanebase + (uint32_t)c0, v);
+              ulonglong2 qv[GP][kBC / 4];
+#pragma unroll
+              for (int j = 0; j < GP; ++j)
+                if (j < G)
+#pragma unroll
+                  for (int e = 0; e < kBC / 4; ++e)
+                    qv[j][e] = *reinterpret_cast<const ulonglong2*>(qs + j * kD + c0 + 4 * e);
+              tmem_wait_ld();
+              if (c0 + kBC == kD) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(BAR_KFREE));
+              }
+#pragma unroll
+              for (int e = 0; e < kBC / 4; ++e) {
+                const uint64_t k01 = pack2(__uint_as_float(v[4 * e + 0]), __uint_as_float(v[4 * e + 1]));
+                const uint64_t k23 = pack2(__uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+#pragma unroll
+                for (int j = 0; j < GP; ++j) {
+                  if (j < G) {
+                    dot[j][(2 * e) % kCh] = ffma2p(k01, qv[j][e].x, dot[j][(2 * e) % kCh]);
+                    dot[j][(2 * e + 1) % kCh] = ffma2p(k23, qv[j][e].y, dot[j][(2 * e + 1) % kCh]);
+                  }
+                }
+              }
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < GP; ++j) {
+#pragma unroll
+            for (int u = 0; u < kCh; ++u) {
+              const float2 d2 = unpack2(dot[j][u]);
+              dsum[j] += d2.x + d2.y;
             }
           }
         }
@@ -540,13 +647,7 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
 #pragma unroll
         for (int j = 0; j < GP; ++j) {
           if (j < G) {
-            float dj = 0.f;
-#pragma unroll
-            for (int u = 0; u < kCh; ++u) {
-              const float2 d2 = unpack2(dot[j][u]);
-              dj += d2.x + d2.y;
-            }
-            sj[j] = valid ? dj * sk : -CUDART_INF_F;
+            sj[j] = valid ? dsum[j] * sk : -CUDART_INF_F;
             const float wm = warp_max(sj[j]);
             if (lane == 0) ms->red[par][j][q4] = wm;
           }
@@ -571,63 +672,132 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
         }
         // ---- value phase: this thread's output dimension ----
         fail = !mbar_wait_warp(bar(BAR_VFULL), ph, abort_flag, kWaitNs);
-        uint32_t v[kBC];
-        if (!fail) {
+        if (!fail && ctid == 0) {
           // MMA1 (KFULL seen) and MMA2 of this tile are complete: their shared-memory
           // operands are free (a commit would only track its own thread's MMAs)
-          if (ctid == 0) {
-            if (!kQuant) mbar_arrive(bar(BAR_EMPTY + (int)(tile_seq % (uint32_t)p.nstage)));
-            else mbar_arrive(bar(BAR_DQEMPTY + (int)(tile_seq & 1u)));
-            if (i == ntiles - 1) mbar_arrive(bar(BAR_BQEMPTY + bx));   // factors and q rows
-          }
-          tc_fence_after();
-          tmem_ld_cols<kBC>(tV + lanebase, v);   // in flight across the barrier
+          if (!kQuant) mbar_arrive(bar(BAR_EMPTY + (int)(tile_seq % (uint32_t)p.nstage)));
+          else mbar_arrive(bar(BAR_DQEMPTY + (int)(tile_seq & 1u)));
+          if (i == ntiles - 1) mbar_arrive(bar(BAR_BQEMPTY + bx));   // factors and q rows
         }
-        const bool stop = bar_any(NB_P, 128, fail);
-        if (stop) {
-          if (!fail) tmem_wait_ld();
-          fail = true;
-          break;
-        }
-#pragma unroll
-        for (int j = 0; j < GP; ++j) {
-          if (j < G) {
-            const uint64_t a2 = pack2(alpha[j], alpha[j]);
-#pragma unroll
-            for (int u = 0; u < kCh; ++u) acc[j][u] = ffma2p(acc[j][u], a2, 0ull);
+        if constexpr (kL16) {
+          uint32_t v0[4 * kN], v1[4 * kN];
+          if (!fail) {
+            tc_fence_after();
+            tmem_ld16x256<kN>(tV + lanebase, v0);   // in flight across the barrier
+            tmem_ld16x256<kN>(tV + lb1, v1);
           }
-        }
-#pragma unroll
-        for (int c0 = 0; c0 < kD; c0 += kBC) {
-          if (c0 > 0) tmem_ld_cols<kBC>(tV + lanebase + (uint32_t)c0, v);
-          ulonglong2 pv[GP][kBC / 4];
-#pragma unroll
-          for (int j = 0; j < GP; ++j)
-            if (j < G)
-#pragma unroll
-              for (int e = 0; e < kBC / 4; ++e)
-                pv[j][e] = *reinterpret_cast<const ulonglong2*>(P + j * kT + c0 + 4 * e);
-          tmem_wait_ld();
-          if (c0 + kBC == kD) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(BAR_VFREE));
-          }
-          if (n_valid < c0 + kBC) {
-            // token columns past the row's length: exact zeros, whatever the cache holds
-#pragma unroll
-            for (int e = 0; e < kBC; ++e)
-              if (c0 + e >= n_valid) v[e] = 0u;
+          const bool stop = bar_any(NB_P, 128, fail);
+          if (stop) {
+            if (!fail) tmem_wait_ld();
+            fail = true;
+            break;
           }
 #pragma unroll
-          for (int e = 0; e < kBC / 4; ++e) {
-            const uint64_t v01 = pack2(__uint_as_float(v[4 * e + 0]), __uint_as_float(v[4 * e + 1]));
-            const uint64_t v23 = pack2(__uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+          for (int j = 0; j < GP; ++j) {
+            if (j < G) {
+              const uint64_t a2 = pack2(alpha[j], alpha[j]);
 #pragma unroll
-            for (int j = 0; j < GP; ++j) {
-              if (j < G) {
-                acc[j][(2 * e) % kCh] = ffma2p(pv[j][e].x, v01, acc[j][(2 * e) % kCh]);
-                acc[j][(2 * e + 1) % kCh] = ffma2p(pv[j][e].y, v23, acc[j][(2 * e + 1) % kCh]);
+              for (int t = 0; t < 4; ++t) acc[t][j] = ffma2p(acc[t][j], a2, 0ull);
+            }
+          }
+#pragma unroll
+          for (int c0 = 0; c0 < kD; c0 += 8 * kN) {
+            if (c0 > 0) {
+              tmem_ld16x256<kN>(tV + lanebase + (uint32_t)c0, v0);
+              tmem_ld16x256<kN>(tV + lb1 + (uint32_t)c0, v1);
+            }
+            uint64_t pp[GP][kN];
+#pragma unroll
+            for (int j = 0; j < GP; ++j)
+              if (j < G)
+#pragma unroll
+                for (int i = 0; i < kN; ++i)
+                  pp[j][i] = *reinterpret_cast<const uint64_t*>(P + j * kT + c0 + 8 * i + 2 * k4);
+            tmem_wait_ld();
+            if (c0 + 8 * kN == kD) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(bar(BAR_VFREE));
+            }
+            if (n_valid < c0 + 8 * kN) {
+              // token columns past the row's length: exact zeros, whatever the cache holds
+#pragma unroll
+              for (int i = 0; i < kN; ++i) {
+                const int col = c0 + 8 * i + 2 * k4;
+                if (col >= n_valid) {
+                  v0[4 * i + 0] = 0u; v0[4 * i + 2] = 0u; v1[4 * i + 0] = 0u; v1[4 * i + 2] = 0u;
+                }
+                if (col + 1 >= n_valid) {
+                  v0[4 * i + 1] = 0u; v0[4 * i + 3] = 0u; v1[4 * i + 1] = 0u; v1[4 * i + 3] = 0u;
+                }
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < kN; ++i) {
+              const uint64_t vp[4] = {
+                  pack2(__uint_as_float(v0[4 * i + 0]), __uint_as_float(v0[4 * i + 1])),
+                  pack2(__uint_as_float(v0[4 * i + 2]), __uint_as_float(v0[4 * i + 3])),
+                  pack2(__uint_as_float(v1[4 * i + 0]), __uint_as_float(v1[4 * i + 1])),
+                  pack2(__uint_as_float(v1[4 * i + 2]), __uint_as_float(v1[4 * i + 3]))};
+#pragma unroll
+              for (int t = 0; t < 4; ++t)
+#pragma unroll
+                for (int j = 0; j < GP; ++j)
+                  if (j < G) acc[t][j] = ffma2p(pp[j][i], vp[t], acc[t][j]);
+            }
+          }
+        } else {
+          uint32_t v[kBC];
+          if (!fail) {
+            tc_fence_after();
+            tmem_ld_cols<kBC>(tV + lanebase, v);   // in flight across the barrier
+          }
+          const bool stop = bar_any(NB_P, 128, fail);
+          if (stop) {
+            if (!fail) tmem_wait_ld();
+            fail = true;
+            break;
+          }
+#pragma unroll
+          for (int j = 0; j < GP; ++j) {
+            if (j < G) {
+              const uint64_t a2 = pack2(alpha[j], alpha[j]);
+#pragma unroll
+              for (int u = 0; u < kCh; ++u) acc[j][u] = ffma2p(acc[j][u], a2, 0ull);
+            }
+          }
+#pragma unroll
+          for (int c0 = 0; c0 < kD; c0 += kBC) {
+            if (c0 > 0) tmem_ld_cols<kBC>(tV + lanebase + (uint32_t)c0, v);
+            ulonglong2 pv[GP][kBC / 4];
+#pragma unroll
+            for (int j = 0; j < GP; ++j)
+              if (j < G)
+#pragma unroll
+                for (int e = 0; e < kBC / 4; ++e)
+                  pv[j][e] = *reinterpret_cast<const ulonglong2*>(P + j * kT + c0 + 4 * e);
+            tmem_wait_ld();
+            if (c0 + kBC == kD) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(bar(BAR_VFREE));
+            }
+            if (n_valid < c0 + kBC) {
+              // token columns past the row's length: exact zeros, whatever the cache holds
+#pragma unroll
+              for (int e = 0; e < kBC; ++e)
+                if (c0 + e >= n_valid) v[e] = 0u;
+            }
+#pragma unroll
+            for (int e = 0; e < kBC / 4; ++e) {
+              const uint64_t v01 = pack2(__uint_as_float(v[4 * e + 0]), __uint_as_float(v[4 * e + 1]));
+              const uint64_t v23 = pack2(__uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+#pragma unroll
+              for (int j = 0; j < GP; ++j) {
+                if (j < G) {
+                  acc[j][(2 * e) % kCh] = ffma2p(pv[j][e].x, v01, acc[j][(2 * e) % kCh]);
+                  acc[j][(2 * e + 1) % kCh] = ffma2p(pv[j][e].y, v23, acc[j][(2 * e + 1) % kCh]);
+                }
               }
             }
           }
@@ -650,10 +820,20 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
           const float4 l4 = *reinterpret_cast<const float4*>(&ms->lsum[j][0]);
           const float L = (l4.x + l4.y) + (l4.z + l4.w);
           float num = 0.f;
+          if constexpr (kL16) {
+            float a4[4];
 #pragma unroll
-          for (int u = 0; u < kCh; ++u) {
-            const float2 a2 = unpack2(acc[j][u]);
-            num += a2.x + a2.y;
+            for (int t = 0; t < 4; ++t) {
+              const float2 a2 = unpack2(acc[t][j]);
+              a4[t] = a2.x + a2.y;
+            }
+            num = reduce_rows4(a4[0], a4[1], a4[2], a4[3], lane);   // output dimension c
+          } else {
+#pragma unroll
+            for (int u = 0; u < kCh; ++u) {
+              const float2 a2 = unpack2(acc[j][u]);
+              num += a2.x + a2.y;
+            }
           }
           a.o_part[((hb + j) * a.S + s) * kD + c] = num / L;
           if (c == j) a.lse_part[(hb + j) * a.S + s] = (m_run[j] + log2f(L)) * CUDART_LN2_F;
