@@ -32,7 +32,7 @@
 //               accumulates P Vhat over the tile's tokens; token columns past the
 //               row's length are zeroed, so cache contents beyond seq_len never reach
 //               the result. At the unit's end it writes the split partial and LSE.
-//   warp 6      (int8 / e4m3 latents only) converts each tile's codes to bf16 (exact)
+//   warps 6-7   (int8 / e4m3 latents only) convert each tile's codes to bf16 (exact)
 //               for MMA1/2; the per-token scales multiply the scores (K) and are
 //               folded into P (V), which is exact algebra.
 // The scores and P V are matrix-vector work (G <= 16 query rows per KV head) and stay
@@ -46,6 +46,7 @@
 // Restrictions: io bf16, latents bf16 / int8 / e4m3, d_head = 128, rank a multiple of
 // 16 in [16, 128], G <= 16, max_seq a multiple of 4 for quantised latents.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <math_constants.h>
 #include <string.h>
@@ -74,8 +75,8 @@ enum LatKind { kLatBF16 = 0, kLatI8 = 1, kLatE4M3 = 2 };
 
 template <int LAT> struct Roles {
   static constexpr int kCons = 2;   // first consumer warp
-  static constexpr int kDQ = 6;     // converter warp (quantised latents)
-  static constexpr int kWarps = LAT == kLatBF16 ? 6 : 7;
+  static constexpr int kDQ = 6;     // converter warps 6, 7 (quantised latents)
+  static constexpr int kWarps = LAT == kLatBF16 ? 6 : 8;
   static constexpr int kThreads = 32 * kWarps;
 };
 
@@ -223,7 +224,7 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
     ms->status_reported = 0;
     for (int i = 0; i < p.nstage; ++i) {
       mbar_init(bar(BAR_FULL + i), 1);
-      mbar_init(bar(BAR_EMPTY + i), 1);
+      mbar_init(bar(BAR_EMPTY + i), kQuant ? 2 : 1);   // converters, or a consumer
     }
     mbar_init(bar(BAR_KFULL), 1);
     mbar_init(bar(BAR_KFREE), 4);
@@ -231,12 +232,12 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
     mbar_init(bar(BAR_VFREE), 4);
     for (int u = 0; u < kUR; ++u) {
       mbar_init(bar(BAR_UFULL + u), 1);
-      mbar_init(bar(BAR_UEMPTY + u), 1 + 4 + (kQuant ? 1 : 0));
+      mbar_init(bar(BAR_UEMPTY + u), 1 + 4 + (kQuant ? 2 : 0));
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar(BAR_BQFULL + x), 1);
       mbar_init(bar(BAR_BQEMPTY + x), 1);   // consumers, after the unit's last MMA2
-      mbar_init(bar(BAR_DQFULL + x), 1);
+      mbar_init(bar(BAR_DQFULL + x), 2);
       mbar_init(bar(BAR_DQEMPTY + x), 1);
       mbar_init(bar(BAR_SCFREE + x), 4);
     }
@@ -844,8 +845,12 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
     if (fail) raise_timeout(a, ms);
   } else if (kQuant && warp >= Roles<LAT>::kDQ) {
     // ============================ code -> bf16 converter ============================
-    // one warp; each thread converts four token rows (lane + 32 k) of the tile
+    // two warps; each thread converts two token rows (rbase, rbase + 64) of the tile.
+    // int8 codes become floats without the int-to-float unit: the biased code byte
+    // is placed in the low mantissa bits of 2^23 and 2^23 + 128 is subtracted (exact);
+    // e4m3 codes convert two at a time through f16 (exact).
     const int W = p.W;
+    const int rbase = (warp - Roles<LAT>::kDQ) * 32 + lane;
     uint32_t tile_seq = 0;
     int unit_seq = 0;
     bool ok = true;
@@ -871,31 +876,36 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
         uint8_t* zop = smem + p.off_zop + (size_t)x * 2u * tile_bytes;
         const float* scs = reinterpret_cast<const float*>(stage + 2 * cb);
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-          const int row = lane + 32 * rr;
+        for (int rr = 0; rr < 2; ++rr) {
+          const int row = rbase + 64 * rr;
 #pragma unroll
           for (int kv = 0; kv < 2; ++kv) {
             const uint8_t* src = stage + kv * cb + (size_t)row * r;
             uint8_t* dst = zop + kv * tile_bytes;
             for (int k0 = 0; k0 < r; k0 += 16) {
               const uint4 raw = *reinterpret_cast<const uint4*>(src + k0);
-              const uint8_t* cbytes = reinterpret_cast<const uint8_t*>(&raw);
+              const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
               uint32_t w[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                float f0, f1;
+              for (int e = 0; e < 4; ++e) {
+                float f[4];
                 if (LAT == kLatI8) {
-                  f0 = (float)(int8_t)cbytes[2 * e];
-                  f1 = (float)(int8_t)cbytes[2 * e + 1];
+                  const uint32_t xb = rw[e] ^ 0x80808080u;   // code + 128, per byte
+                  f[0] = __int_as_float((int)__byte_perm(xb, 0x4B000000u, 0x7540u)) - 8388736.f;
+                  f[1] = __int_as_float((int)__byte_perm(xb, 0x4B000000u, 0x7541u)) - 8388736.f;
+                  f[2] = __int_as_float((int)__byte_perm(xb, 0x4B000000u, 0x7542u)) - 8388736.f;
+                  f[3] = __int_as_float((int)__byte_perm(xb, 0x4B000000u, 0x7543u)) - 8388736.f;
                 } else {
-                  __nv_fp8_e4m3 c0, c1;
-                  c0.__x = cbytes[2 * e];
-                  c1.__x = cbytes[2 * e + 1];
-                  f0 = (float)c0;
-                  f1 = (float)c1;
+                  const __half2_raw h01 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(rw[e] & 0xFFFFu), __NV_E4M3);
+                  const __half2_raw h23 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(rw[e] >> 16), __NV_E4M3);
+                  const float2 a01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+                  const float2 a23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+                  f[0] = a01.x; f[1] = a01.y; f[2] = a23.x; f[3] = a23.y;
                 }
-                const __nv_bfloat162 bb = __floats2bfloat162_rn(f0, f1);
-                w[e] = *reinterpret_cast<const uint32_t*>(&bb);
+                const __nv_bfloat162 b01 = __floats2bfloat162_rn(f[0], f[1]);
+                const __nv_bfloat162 b23 = __floats2bfloat162_rn(f[2], f[3]);
+                w[2 * e] = *reinterpret_cast<const uint32_t*>(&b01);
+                w[2 * e + 1] = *reinterpret_cast<const uint32_t*>(&b23);
               }
               // bf16 bytes [2*k0, 2*k0 + 32) of this row: two 16-byte chunks, swizzled
 #pragma unroll
