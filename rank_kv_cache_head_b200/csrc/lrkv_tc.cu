@@ -113,7 +113,13 @@ __device__ __forceinline__ float reduce_rows4(float a0, float a1, float a2, floa
 }
 
 // named barriers of the consumer warpgroup (id 0 is __syncthreads)
-enum { NB_Q = 1, NB_MAX = 2, NB_P = 3, NB_END = 4 };
+enum { NB_Q = 1, NB_MAX = 2, NB_P = 3, NB_END = 4, NB_RED = 5 };
+
+// 16x256b consumers keep a reference max per head and weight a tile's tokens by
+// 2^(s - reference) with no per-tile max exchange; only a tile with a score above the
+// reference by more than kTau (log2 units) moves it (an exact rescale). Weights stay
+// below 2^kTau, far from fp32 overflow.
+constexpr float kTau = 8.f;
 
 struct alignas(64) TcParams {
   CUtensorMap tm_zk, tm_zv, tm_bk, tm_bv, tm_sk, tm_sv;
@@ -645,30 +651,49 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
           }
         }
         float sj[GP];
-#pragma unroll
-        for (int j = 0; j < GP; ++j) {
-          if (j < G) {
-            sj[j] = valid ? dsum[j] * sk : -CUDART_INF_F;
-            const float wm = warp_max(sj[j]);
-            if (lane == 0) ms->red[par][j][q4] = wm;
-          }
-        }
-        if (bar_any(NB_MAX, 128, fail)) { fail = true; break; }
-        // ---- online softmax over the tile: one running max per head ----
         float* P = ps_all + par * (G * kT);
         float alpha[GP];
+        float pfin[GP];      // this thread's weight per head (added to the running sum)
+        bool over = false;   // 16x256b: a score above the reference max + kTau
+        if constexpr (kL16) {
 #pragma unroll
-        for (int j = 0; j < GP; ++j) {
-          alpha[j] = 1.f;
-          if (j < G) {
-            const float4 wm = *reinterpret_cast<const float4*>(&ms->red[par][j][0]);
-            const float m_new = fmaxf(m_run[j], fmaxf(fmaxf(wm.x, wm.y), fmaxf(wm.z, wm.w)));
-            alpha[j] = (m_new == -CUDART_INF_F) ? 1.f : exp2f(m_run[j] - m_new);
-            const float pj = valid ? exp2f(sj[j] - m_new) : 0.f;
-            l_run[j] = l_run[j] * alpha[j] + pj;
-            m_run[j] = m_new;
-            // masked tokens contribute an exact zero (their scale may be anything)
-            P[j * kT + row] = valid ? pj * sv : 0.f;
+          for (int j = 0; j < GP; ++j) {
+            alpha[j] = 1.f;
+            pfin[j] = 0.f;
+            sj[j] = -CUDART_INF_F;
+            if (j < G) {
+              sj[j] = valid ? dsum[j] * sk : -CUDART_INF_F;
+              over = over || (sj[j] > m_run[j] + kTau);
+              const float pj = valid ? exp2f(sj[j] - m_run[j]) : 0.f;
+              pfin[j] = pj;
+              // masked tokens contribute an exact zero (their scale may be anything)
+              P[j * kT + row] = valid ? pj * sv : 0.f;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < GP; ++j) {
+            if (j < G) {
+              sj[j] = valid ? dsum[j] * sk : -CUDART_INF_F;
+              const float wm = warp_max(sj[j]);
+              if (lane == 0) ms->red[par][j][q4] = wm;
+            }
+          }
+          if (bar_any(NB_MAX, 128, fail)) { fail = true; break; }
+          // ---- online softmax over the tile: one running max per head ----
+#pragma unroll
+          for (int j = 0; j < GP; ++j) {
+            alpha[j] = 1.f;
+            if (j < G) {
+              const float4 wm = *reinterpret_cast<const float4*>(&ms->red[par][j][0]);
+              const float m_new = fmaxf(m_run[j], fmaxf(fmaxf(wm.x, wm.y), fmaxf(wm.z, wm.w)));
+              alpha[j] = (m_new == -CUDART_INF_F) ? 1.f : exp2f(m_run[j] - m_new);
+              const float pj = valid ? exp2f(sj[j] - m_new) : 0.f;
+              l_run[j] = l_run[j] * alpha[j] + pj;
+              m_run[j] = m_new;
+              // masked tokens contribute an exact zero (their scale may be anything)
+              P[j * kT + row] = valid ? pj * sv : 0.f;
+            }
           }
         }
         // ---- value phase: this thread's output dimension ----
@@ -687,20 +712,48 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
             tmem_ld16x256<kN>(tV + lanebase, v0);   // in flight across the barrier
             tmem_ld16x256<kN>(tV + lb1, v1);
           }
-          const bool stop = bar_any(NB_P, 128, fail);
-          if (stop) {
-            if (!fail) tmem_wait_ld();
-            fail = true;
-            break;
-          }
+          // P of the tile complete; the barrier also ORs in a failed wait or a score
+          // above the reference max
+          const bool rare = bar_any(NB_P, 128, fail || over);
+          if (rare) {
+            if (bar_any(NB_MAX, 128, fail)) {
+              if (!fail) tmem_wait_ld();
+              fail = true;
+              break;
+            }
+            // move the reference to the tile's max, rescale, and rewrite the tile's P
 #pragma unroll
-          for (int j = 0; j < GP; ++j) {
-            if (j < G) {
-              const uint64_t a2 = pack2(alpha[j], alpha[j]);
+            for (int j = 0; j < GP; ++j) {
+              if (j < G) {
+                const float wm = warp_max(sj[j]);
+                if (lane == 0) ms->red[par][j][q4] = wm;
+              }
+            }
+            bar_any(NB_RED, 128, false);
 #pragma unroll
-              for (int t = 0; t < 4; ++t) acc[t][j] = ffma2p(acc[t][j], a2, 0ull);
+            for (int j = 0; j < GP; ++j) {
+              if (j < G) {
+                const float4 wm = *reinterpret_cast<const float4*>(&ms->red[par][j][0]);
+                const float m_new = fmaxf(m_run[j], fmaxf(fmaxf(wm.x, wm.y), fmaxf(wm.z, wm.w)));
+                alpha[j] = (m_new == -CUDART_INF_F) ? 1.f : exp2f(m_run[j] - m_new);
+                pfin[j] = valid ? exp2f(sj[j] - m_new) : 0.f;
+                m_run[j] = m_new;
+                P[j * kT + row] = valid ? pfin[j] * sv : 0.f;
+              }
+            }
+            bar_any(NB_RED, 128, false);
+#pragma unroll
+            for (int j = 0; j < GP; ++j) {
+              if (j < G) {
+                const uint64_t a2 = pack2(alpha[j], alpha[j]);
+#pragma unroll
+                for (int t = 0; t < 4; ++t) acc[t][j] = ffma2p(acc[t][j], a2, 0ull);
+              }
             }
           }
+#pragma unroll
+          for (int j = 0; j < GP; ++j)
+            if (j < G) l_run[j] = l_run[j] * alpha[j] + pfin[j];
 #pragma unroll
           for (int c0 = 0; c0 < kD; c0 += 8 * kN) {
             if (c0 > 0) {
