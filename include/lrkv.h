@@ -223,6 +223,19 @@ int lrkv_decode_attn_noalloc(const lrkv_dims* dims, const void* q, const void* Z
                              float* lse_out, uint32_t* status_out, void* stream);
 
 /*
+ * Test hook for the bounded-wait error path (the paper has no counterpart). With on
+ * != 0, the next tensor-core split launch (and only that one) runs with the producer
+ * of the CTA that takes work unit 0 withholding the copy and the arrival of that
+ * unit's first latent tile: the mbarrier waits on that tile run out after their
+ * one-second bound, that CTA unwinds
+ * (it drains its own copies and MMAs and frees its tensor memory) and the launch
+ * sets LRKV_STATUS_TIMEOUT in the workspace status word; the other CTAs finish
+ * normally and the context stays usable. Outputs of such a launch are not valid.
+ * Returns 0.
+ */
+int lrkv_debug_stall_next_launch(int32_t on);
+
+/*
  * Synchronise stream, copy the workspace status word to *status and clear it.
  * Returns 0, or LRKV_ERR_LAUNCH if the copy failed.
  */

@@ -4,6 +4,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <functional>
 #include <map>
 #include <mutex>
@@ -31,6 +32,9 @@ int num_sms() {
 }
 
 namespace {
+
+// set by lrkv_debug_stall_next_launch, consumed by the next tensor-core launch
+std::atomic<int> g_debug_stall{0};
 
 size_t dtype_bytes(int t) { return t == LRKV_F32 ? 4 : (t == LRKV_BF16 ? 2 : 1); }
 
@@ -260,6 +264,7 @@ int lrkv_decode_attn_timed(const lrkv_dims* dims, const void* q, const void* ZK,
   a.io_dtype = dims->io_dtype;
   a.latent_dtype = dims->latent_dtype;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_head));
+  a.debug_stall = 0;
 
   if (p.algo == LRKV_ALGO_TCGEN05 && quant &&
       ((reinterpret_cast<uintptr_t>(ZK_scale) | reinterpret_cast<uintptr_t>(ZV_scale)) & 15u)) {
@@ -268,6 +273,7 @@ int lrkv_decode_attn_timed(const lrkv_dims* dims, const void* q, const void* ZK,
     p.smem = (int)simt_smem_bytes(dims->rank, dims->d_head, dims->n_q_heads / dims->n_kv_heads);
     if (p.smem > 227 * 1024) return LRKV_ERR_UNSUPPORTED;
   }
+  if (p.algo == LRKV_ALGO_TCGEN05) a.debug_stall = g_debug_stall.exchange(0);
   record_event(ev_split_begin, st);
   cudaError_t e = (p.algo == LRKV_ALGO_TCGEN05) ? launch_split_tc(a, p, st)
                                                 : launch_split_simt(a, p, st);
@@ -349,6 +355,11 @@ int lrkv_decode_step_host(const lrkv_dims* dims, const void* q_host, const void*
   if (rc) return rc;
   if (cudaMemcpyAsync(out_host, out_dev, qbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
     return LRKV_ERR_LAUNCH;
+  return LRKV_OK;
+}
+
+int lrkv_debug_stall_next_launch(int32_t on) {
+  g_debug_stall.store(on ? 1 : 0);
   return LRKV_OK;
 }
 

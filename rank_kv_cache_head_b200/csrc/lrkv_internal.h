@@ -45,6 +45,7 @@ struct SplitArgs {
   int B, Hq, Hkv, G, d, r, Lcap, max_seqlen, S, chunk;
   int io_dtype, latent_dtype;
   float scale_log2;  // log2(e) / sqrt(d)
+  int debug_stall;   // test hook: work unit 0's first tile is withheld (see lrkv.h)
 };
 
 struct MergeArgs {

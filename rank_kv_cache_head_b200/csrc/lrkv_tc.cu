@@ -346,7 +346,10 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
           ok = false;
           break;
         }
-        if (leader) {
+        // test hook: the CTA that took work unit 0 withholds that unit's first tile (copy
+        // and arrival), so the waits on it run out and the bounded-wait error path runs
+        const bool withhold = a.debug_stall && u == 0 && i == 0;
+        if (leader && !withhold) {
           const uint32_t sst = sbase + p.off_stage + (uint32_t)st * p.stage_bytes;
           const int row = row0 + i * kT;
           if (!kQuant) {

@@ -78,6 +78,7 @@ def lib() -> ctypes.CDLL:
         L.lrkv_decode_attn_noalloc.argtypes = [dp] + [_vp] * 12
         L.lrkv_decode_step_host.argtypes = [dp] + [_vp] * 16 + [ctypes.c_size_t, _vp]
         L.lrkv_read_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
+        L.lrkv_debug_stall_next_launch.argtypes = [ctypes.c_int32]
         _lib = L
     return _lib
 
@@ -207,6 +208,13 @@ def decode_attn_noalloc(dims: Dims, q, ZK, ZV, ZK_scale, ZV_scale, BK, BV, seqle
     rc = lib().lrkv_decode_attn_noalloc(ctypes.byref(dims), *args, _stream(stream))
     if rc:
         raise LrkvError("lrkv_decode_attn_noalloc", rc)
+
+
+def debug_stall_next_launch(on: bool = True) -> None:
+    """Test hook: the next tensor-core split launch withholds the first tile of work
+    unit 0 so the waits on it run out (LRKV_STATUS_TIMEOUT); see
+    lrkv_debug_stall_next_launch."""
+    lib().lrkv_debug_stall_next_launch(1 if on else 0)
 
 
 class PreparedStep:
