@@ -198,6 +198,27 @@ int lrkv_decode_step_host(const lrkv_dims* dims, const void* q_host, const void*
                           size_t workspace_bytes, void* stream);
 
 /*
+ * Fused latent projection + append, the step that produces the row lrkv_append
+ * writes ("WSVD: Weighted Low-Rank Approximation for Fast and Efficient Execution of
+ * Low-Precision Vision-Language Models", section 2.A: the cached latent of a head is
+ * the token's hidden state times that head's down factor A, W = A B). For every batch
+ * row b and KV head g:
+ *     z_K = x[b] . AK[g],   z_V = x[b] . AV[g]     (fp32 accumulation)
+ * written at slot seqlens[b] exactly as lrkv_append writes a row (fp32, bf16 RNE, or
+ * int8 / e4m3 codes with a per-row fp32 absmax scale), then seqlens[b] += 1.
+ *   x      [B][d_model], io dtype, device
+ *   AK, AV [H_kv][d_model][rank], io dtype, device
+ *   other arguments as lrkv_append (workspace: its header, >= 256 bytes).
+ * Errors: LRKV_ERR_DIMS (dims, d_model outside [1, 2^20]), LRKV_ERR_ARG (NULL pointer,
+ * scales present iff quantised latents), LRKV_ERR_ALIGN, LRKV_ERR_WORKSPACE,
+ * LRKV_ERR_LAUNCH. A row whose slot is past the capacity is left untouched, keeps its
+ * length and sets LRKV_STATUS_APPEND_FULL.
+ */
+int lrkv_project_append(const lrkv_dims* dims, int32_t d_model, const void* x, const void* AK,
+                        const void* AV, void* ZK, void* ZV, float* ZK_scale, float* ZV_scale,
+                        int32_t* seqlens, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Decode attention for callers that cannot allocate device memory (a host program
  * without a device memory manager, or a runtime whose memory budget forbids new
  * allocations while it serves). The paper has no counterpart: this is a deployment

@@ -335,3 +335,23 @@ def append(ZK, ZV, ZK_scale, ZV_scale, seqlens, zk_new32, zv_new32, latent_dtype
                     raise ValueError(latent_dtype)
         seqlens[b] = slot + 1
     return ZK, ZV, ZK_scale, ZV_scale, seqlens, status
+
+
+def project(x, AK, AV):
+    """The new token's latents for every (batch row, KV head): z_K = x A_K,g and
+    z_V = x A_V,g (the cached latent is the token's hidden state times the head's down
+    factor, W = A B: "WSVD: Weighted Low-Rank Approximation for Fast and Efficient
+    Execution of Low-Precision Vision-Language Models", section 2.A), in fp64.
+    x [B][d_model], A [Hkv][d_model][r] -> two arrays [B][Hkv][r]."""
+    x = np.asarray(x, np.float64)
+    AK = np.asarray(AK, np.float64)
+    AV = np.asarray(AV, np.float64)
+    return np.einsum("bi,gir->bgr", x, AK), np.einsum("bi,gir->bgr", x, AV)
+
+
+def project_append(ZK, ZV, ZK_scale, ZV_scale, seqlens, x, AK, AV, latent_dtype: str):
+    """Fused projection + append: project, take the fp32 value of each latent (the
+    precision the kernel stores and quantises in), then append as above."""
+    zk, zv = project(x, AK, AV)
+    return append(ZK, ZV, ZK_scale, ZV_scale, seqlens, zk.astype(np.float32),
+                  zv.astype(np.float32), latent_dtype)

@@ -328,6 +328,40 @@ int lrkv_append(const lrkv_dims* dims, const void* zk_new, const void* zv_new, v
   return LRKV_OK;
 }
 
+int lrkv_project_append(const lrkv_dims* dims, int32_t d_model, const void* x, const void* AK,
+                        const void* AV, void* ZK, void* ZV, float* ZK_scale, float* ZV_scale,
+                        int32_t* seqlens, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (d_model < 1 || d_model > (1 << 20)) return LRKV_ERR_DIMS;
+  const bool quant = dims->latent_dtype == LRKV_I8 || dims->latent_dtype == LRKV_E4M3;
+  if (!x || !AK || !AV || !ZK || !ZV || !seqlens || !workspace) return LRKV_ERR_ARG;
+  if (quant != (ZK_scale != nullptr) || quant != (ZV_scale != nullptr)) return LRKV_ERR_ARG;
+  if (workspace_bytes < kHeaderBytes) return LRKV_ERR_WORKSPACE;
+  if (!aligned16(ZK) || !aligned16(ZV) || !aligned16(workspace)) return LRKV_ERR_ALIGN;
+  ProjArgs a;
+  a.app.zk_new = nullptr;
+  a.app.zv_new = nullptr;
+  a.app.ZK = ZK;
+  a.app.ZV = ZV;
+  a.app.SK = ZK_scale;
+  a.app.SV = ZV_scale;
+  a.app.seqlens = seqlens;
+  a.app.header = static_cast<uint32_t*>(workspace);
+  a.app.B = dims->batch;
+  a.app.Hkv = dims->n_kv_heads;
+  a.app.r = dims->rank;
+  a.app.Lcap = dims->max_seq;
+  a.app.io_dtype = dims->io_dtype;
+  a.app.latent_dtype = dims->latent_dtype;
+  a.x = x;
+  a.AK = AK;
+  a.AV = AV;
+  a.d_model = d_model;
+  if (launch_project_append(a, (cudaStream_t)stream) != cudaSuccess) return LRKV_ERR_LAUNCH;
+  return LRKV_OK;
+}
+
 int lrkv_decode_step_host(const lrkv_dims* dims, const void* q_host, const void* zk_new_host,
                           const void* zv_new_host, void* out_host, void* q_dev,
                           void* zk_new_dev, void* zv_new_dev, void* out_dev, void* ZK, void* ZV,

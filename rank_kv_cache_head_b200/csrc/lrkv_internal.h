@@ -15,7 +15,7 @@ constexpr int kTile = 128;            // tokens per pipeline tile / split granul
 constexpr size_t kHeaderBytes = 256;  // workspace header: status word + counters
 
 // Workspace header words.
-enum HeaderWord { kStatusWord = 0, kWorkCounter = 1, kDoneCounter = 2 };
+enum HeaderWord { kStatusWord = 0, kWorkCounter = 1, kDoneCounter = 2, kProjCounter = 3 };
 
 // Launch plan for one call (depends only on dims and the device).
 struct Plan {
@@ -72,6 +72,16 @@ struct AppendArgs {
   int io_dtype, latent_dtype;
 };
 
+// The fused latent projection + append: the new token's latents z = x A_g are
+// computed here instead of being passed in.
+struct ProjArgs {
+  AppendArgs app;   // zk_new / zv_new unused
+  const void* x;    // [B][d_model], io dtype
+  const void* AK;   // [Hkv][d_model][r], io dtype
+  const void* AV;
+  int d_model;
+};
+
 // Programmatic dependent launch: every kernel of the library is launched so that it
 // may start while the previous kernel of the stream finishes, and waits for that
 // kernel (and so, transitively, every earlier one) before it touches memory they
@@ -104,6 +114,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 cudaError_t launch_split_simt(const SplitArgs& a, const Plan& p, cudaStream_t st);
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t st);
+cudaError_t launch_project_append(const ProjArgs& a, cudaStream_t st);
 
 // tcgen05 path: whether it supports these dims, its shared memory per CTA and CTAs
 // per SM, and the launcher.

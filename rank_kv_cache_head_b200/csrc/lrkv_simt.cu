@@ -330,6 +330,103 @@ __global__ void __launch_bounds__(1024) lrkv_append_kernel(AppendArgs a) {
   if (threadIdx.x == 0) a.seqlens[b] = slot + 1;
 }
 
+
+// Fused latent projection + append (the step before decode attention): for every
+// batch row b and KV head g, the new token's latents z_K = x_b A_K,g and
+// z_V = x_b A_V,g ("WSVD: Weighted Low-Rank Approximation for Fast and Efficient
+// Execution of Low-Precision Vision-Language Models", section 2.A: the cached latent
+// is the token's hidden state times the down factor), accumulated in fp32 and
+// written at slot seqlens[b] exactly as lrkv_append writes a row (bf16 RNE, or int8 /
+// e4m3 codes with a per-row absmax scale). The last CTA to finish advances seqlens.
+// grid (2 Hkv): CTA = (KV head, K | V); 256 threads = column k (t % r) x row group
+// (t / r). It reads its factor once per group of 16 batch rows (later groups from
+// L2), with the rows of x staged in shared memory 256 columns at a time.
+constexpr int kProjThreads = 256;
+constexpr int kProjRows = 16;     // batch rows per pass (accumulators a thread)
+constexpr int kProjChunk = 256;   // columns of x staged per step
+
+template <int LAT>
+__global__ void __launch_bounds__(kProjThreads) lrkv_project_append_kernel(ProjArgs pa) {
+  __shared__ float xs[kProjRows * kProjChunk];
+  __shared__ float red[kProjThreads * kProjRows];   // [row group][batch row][column]
+  __shared__ float zs[kProjRows * 256];
+  griddep_wait();
+  griddep_launch_dependents();
+  const AppendArgs& a = pa.app;
+  const int g = blockIdx.x >> 1, kv = blockIdx.x & 1;
+  const int r = a.r, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int ngr = kProjThreads / r;                 // row groups (r divides into 256 or not)
+  const int k = t % r, rg = t / r;
+  const bool active = rg < ngr;
+  const int D = pa.d_model;
+  const void* A = kv ? pa.AV : pa.AK;
+  const size_t abase = (size_t)g * D * r;
+  for (int b0 = 0; b0 < a.B; b0 += kProjRows) {
+    const int nb = min(kProjRows, a.B - b0);
+    float acc[kProjRows];
+#pragma unroll
+    for (int bb = 0; bb < kProjRows; ++bb) acc[bb] = 0.f;
+    for (int d0 = 0; d0 < D; d0 += kProjChunk) {
+      __syncthreads();
+      for (int idx = t; idx < kProjRows * kProjChunk; idx += kProjThreads) {
+        const int bb = idx / kProjChunk, dd = idx - bb * kProjChunk;
+        xs[idx] = (bb < nb && d0 + dd < D) ? load_io(pa.x, (size_t)(b0 + bb) * D + d0 + dd, a.io_dtype) : 0.f;
+      }
+      __syncthreads();
+      if (active) {
+        const int dn = min(kProjChunk, D - d0);
+        for (int i = rg; i < dn; i += ngr) {
+          const float av = load_io(A, abase + (size_t)(d0 + i) * r + k, a.io_dtype);
+#pragma unroll
+          for (int bb = 0; bb < kProjRows; ++bb) acc[bb] = fmaf(xs[bb * kProjChunk + i], av, acc[bb]);
+        }
+      }
+    }
+    __syncthreads();
+    if (active) {
+#pragma unroll
+      for (int bb = 0; bb < kProjRows; ++bb) red[(rg * kProjRows + bb) * r + k] = acc[bb];
+    }
+    __syncthreads();
+    // the row groups' partial sums in a fixed order
+    for (int idx = t; idx < nb * r; idx += kProjThreads) {
+      const int bb = idx / r, kk = idx - bb * r;
+      float z = 0.f;
+      for (int q = 0; q < ngr; ++q) z += red[(q * kProjRows + bb) * r + kk];
+      zs[bb * r + kk] = z;
+    }
+    __syncthreads();
+    // one warp per batch row writes the row (and its scale) at the row's slot
+    for (int bb = warp; bb < nb; bb += kProjThreads / 32) {
+      const int b = b0 + bb;
+      const int slot = a.seqlens[b];
+      if (slot < 0 || slot >= a.Lcap) {
+        if (lane == 0) atomicOr(a.header + kStatusWord, LRKV_STATUS_APPEND_FULL);
+        continue;
+      }
+      float zz[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) zz[e] = (lane + 32 * e < r) ? zs[bb * r + lane + 32 * e] : 0.f;
+      append_row<LAT>(a, b, 2 * g + kv, slot, lane, zz);
+    }
+  }
+  // the last CTA to finish advances every valid row's length (all CTAs have read it)
+  __syncthreads();
+  if (t == 0) {
+    __threadfence();
+    const unsigned prev = atomicAdd(a.header + kProjCounter, 1u);
+    if (prev == gridDim.x - 1) {
+      __threadfence();
+      for (int b = 0; b < a.B; ++b) {
+        const int slot = a.seqlens[b];
+        if (slot >= 0 && slot < a.Lcap) a.seqlens[b] = slot + 1;
+      }
+      atomicExch(a.header + kProjCounter, 0u);
+      __threadfence();
+    }
+  }
+}
+
 }  // namespace
 
 size_t simt_smem_bytes(int r, int d, int G) {
@@ -369,6 +466,16 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t st) {
     case LRKV_BF16: return launch_pdl(lrkv_append_kernel<LRKV_BF16>, dim3(a.B), dim3(threads), 0, st, a);
     case LRKV_I8: return launch_pdl(lrkv_append_kernel<LRKV_I8>, dim3(a.B), dim3(threads), 0, st, a);
     default: return launch_pdl(lrkv_append_kernel<LRKV_E4M3>, dim3(a.B), dim3(threads), 0, st, a);
+  }
+}
+
+cudaError_t launch_project_append(const ProjArgs& a, cudaStream_t st) {
+  const dim3 grid(2 * a.app.Hkv), block(kProjThreads);
+  switch (a.app.latent_dtype) {
+    case LRKV_F32: return launch_pdl(lrkv_project_append_kernel<LRKV_F32>, grid, block, 0, st, a);
+    case LRKV_BF16: return launch_pdl(lrkv_project_append_kernel<LRKV_BF16>, grid, block, 0, st, a);
+    case LRKV_I8: return launch_pdl(lrkv_project_append_kernel<LRKV_I8>, grid, block, 0, st, a);
+    default: return launch_pdl(lrkv_project_append_kernel<LRKV_E4M3>, grid, block, 0, st, a);
   }
 }
 

@@ -79,6 +79,7 @@ def lib() -> ctypes.CDLL:
         L.lrkv_decode_step_host.argtypes = [dp] + [_vp] * 16 + [ctypes.c_size_t, _vp]
         L.lrkv_read_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
         L.lrkv_debug_stall_next_launch.argtypes = [ctypes.c_int32]
+        L.lrkv_project_append.argtypes = [dp, ctypes.c_int32] + [_vp] * 9 + [ctypes.c_size_t, _vp]
         _lib = L
     return _lib
 
@@ -265,6 +266,25 @@ def append(dims: Dims, zk_new, zv_new, ZK, ZV, ZK_scale, ZV_scale, seqlens, work
     rc = lib().lrkv_append(ctypes.byref(dims), *args, workspace.numel(), _stream(stream))
     if rc:
         raise LrkvError("lrkv_append", rc)
+
+
+def project_append(dims: Dims, x, AK, AV, ZK, ZV, ZK_scale, ZV_scale, seqlens, workspace,
+                   stream=None) -> None:
+    """lrkv_project_append: z = x A_g for every (b, KV head), written at seqlens[b] as
+    lrkv_append writes a row, then seqlens[b] += 1. x [B][d_model], A [Hkv][d_model][r]."""
+    sh = _shapes(dims)
+    io = sh["q"][1]
+    d_model = x.numel() // dims.batch if x is not None else 0
+    args = [_ptr(x, "x", io, dims.batch * d_model),
+            _ptr(AK, "AK", io, dims.n_kv_heads * d_model * dims.rank),
+            _ptr(AV, "AV", io, dims.n_kv_heads * d_model * dims.rank),
+            _ptr(ZK, "ZK", *sh["Z"][::-1]), _ptr(ZV, "ZV", *sh["Z"][::-1]),
+            _ptr(ZK_scale, "ZK_scale", *sh["S"][::-1]), _ptr(ZV_scale, "ZV_scale", *sh["S"][::-1]),
+            _ptr(seqlens, "seqlens", *sh["seq"][::-1]), _ptr(workspace, "workspace")]
+    rc = lib().lrkv_project_append(ctypes.byref(dims), d_model, *args, workspace.numel(),
+                                   _stream(stream))
+    if rc:
+        raise LrkvError("lrkv_project_append", rc)
 
 
 def decode_step_host(dims: Dims, q_host, zk_new_host, zv_new_host, out_host, q_dev, zk_new_dev,

@@ -1,0 +1,93 @@
+"""GPU parity of the fused latent projection + append (lrkv_project_append) against
+the oracle: the row lengths advance exactly (a full row keeps its length and sets the
+status bit), every cache entry other than the appended ones is untouched, and the
+appended latents match the oracle's projection stored the same way. The kernel
+accumulates in fp32 where the oracle uses fp64, so a stored value may differ by one
+rounding step of the stored format where the exact value sits next to a boundary."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import lrkv_oracle as orc
+from rank_kv_cache_head_b200 import lrkv
+from rank_kv_cache_head_b200.workloads import stored_bits
+
+pytestmark = pytest.mark.gpu
+
+_IO = {"f32": torch.float32, "bf16": torch.bfloat16}
+_LAT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def _decode(bits, lat):
+    return orc.decode_stored(bits, lat)
+
+
+@pytest.mark.parametrize("io,lat,r,D", [("f32", "f32", 32, 300), ("bf16", "bf16", 32, 300),
+                                        ("bf16", "bf16", 48, 1000), ("bf16", "i8", 32, 520),
+                                        ("bf16", "e4m3", 64, 256)])
+def test_project_append_matches_oracle(io, lat, r, D):
+    B, H, Lcap = 3, 2, 64
+    rng = np.random.default_rng(1000 + r + D)
+    x = torch.from_numpy(rng.standard_normal((B, D))).to(_IO[io])
+    AK = torch.from_numpy(rng.standard_normal((H, D, r)) / math.sqrt(D)).to(_IO[io])
+    AV = torch.from_numpy(rng.standard_normal((H, D, r)) / math.sqrt(D)).to(_IO[io])
+    Z0 = torch.from_numpy(rng.standard_normal((2, B, H, Lcap, r)) * (30 if lat in ("i8", "e4m3") else 1))
+    if lat == "i8":
+        Z0 = Z0.clamp(-127, 127).round().to(torch.int8)
+    elif lat == "e4m3":
+        Z0 = Z0.clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)   # stored codes
+    else:
+        Z0 = Z0.to(_LAT[lat])
+    quant = lat in ("i8", "e4m3")
+    S0 = torch.from_numpy(rng.uniform(0.5, 1.5, (2, B, H, Lcap)).astype(np.float32)) if quant else None
+    seq0 = torch.tensor([5, Lcap - 1, Lcap], dtype=torch.int32)
+
+    dims = lrkv.make_dims(B, H, H, 128, r, Lcap, Lcap, io, lat)
+    ZK, ZV = Z0[0].clone().cuda(), Z0[1].clone().cuda()
+    SK = None if S0 is None else S0[0].clone().cuda()
+    SV = None if S0 is None else S0[1].clone().cuda()
+    seq = seq0.clone().cuda()
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    lrkv.project_append(dims, x.cuda(), AK.cuda(), AV.cuda(), ZK, ZV, SK, SV, seq, ws)
+    status = lrkv.read_status(ws)
+    assert status & lrkv.STATUS_APPEND_FULL
+
+    f64 = lambda t: t.double().numpy()
+    ref = orc.project_append(stored_bits(Z0[0]), stored_bits(Z0[1]),
+                             None if S0 is None else S0[0].numpy(), None if S0 is None else S0[1].numpy(),
+                             seq0.numpy(), f64(x), f64(AK), f64(AV), lat)
+    rZK, rZV, rSK, rSV, rseq, rst = ref
+    assert rst & orc.STATUS_APPEND_FULL
+    np.testing.assert_array_equal(seq.cpu().numpy(), rseq)
+
+    for got_t, want_bits, init_bits, got_s, want_s in (
+            (ZK, rZK, stored_bits(Z0[0]), SK, rSK), (ZV, rZV, stored_bits(Z0[1]), SV, rSV)):
+        got_bits = stored_bits(got_t.cpu())
+        mask = np.zeros(got_bits.shape[:3], bool)        # appended (b, g, slot) entries
+        for b in range(B):
+            if 0 <= int(seq0[b]) < Lcap:
+                mask[b, :, int(seq0[b])] = True
+        # everything else untouched, bit for bit
+        np.testing.assert_array_equal(got_bits[~mask], init_bits[~mask])
+        if quant:
+            np.testing.assert_array_equal(got_s.cpu().numpy()[~mask], S0.numpy()[0 if got_t is ZK else 1][~mask])
+        got_v = _decode(got_bits[mask], lat)
+        want_v = _decode(want_bits[mask], lat)
+        if lat == "f32":
+            np.testing.assert_allclose(got_v, want_v, rtol=1e-5, atol=1e-6)
+        elif lat == "bf16":
+            # at most one bf16 step (2^-7 relative) apart
+            assert np.all(np.abs(got_v - want_v) <= np.abs(want_v) * 2.0 ** -7 + 1e-30)
+        else:
+            gs, ws_ = got_s.cpu().numpy()[mask], want_s[mask]
+            np.testing.assert_allclose(gs, ws_, rtol=1e-5)
+            # codes: one rounding step at most, and almost all identical
+            diff = np.abs(got_v - want_v)
+            assert np.mean(diff == 0) >= 0.97
+            if lat == "i8":
+                assert diff.max() <= 1.0
+            else:
+                # neighbouring e4m3 codes: relative gap 2^-3 in the normal range
+                assert np.all(diff <= np.maximum(np.abs(want_v) * 2.0 ** -3, 2.0 ** -9) + 1e-30)
