@@ -65,6 +65,8 @@ def parse():
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--projection-dmodel", type=int, default=4096,
+                    help="also time lrkv_project_append with this hidden size (0: skip)")
     ap.add_argument("--profile", type=int, default=0, metavar="N",
                     help="no timing: run N eager decode-attention calls on one cache copy "
                          "and exit (a short, fixed launch sequence for ncu captures)")
@@ -104,10 +106,16 @@ def barrier():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the split kernel's sources (the kernel file and the headers it includes):
+    DRAM counters taken on other sources do not describe it."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "rank_kv_cache_head_b200", "csrc", "*"))):
-        with open(p, "rb") as f:
-            h.update(os.path.basename(p).encode() + f.read())
+    csrc = os.path.join(ROOT, "rank_kv_cache_head_b200", "csrc")
+    for name in ("lrkv_tc.cu", "lrkv_sm100.cuh", "lrkv_tmap.h", "lrkv_internal.h"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    inc = os.path.join(ROOT, "include", "lrkv.h")
+    with open(inc, "rb") as f:
+        h.update(b"lrkv.h" + f.read())
     return h.hexdigest()[:16]
 
 
@@ -246,6 +254,65 @@ def largest_divisor_at_most(k: int, cap: int) -> int:
         if k % g == 0:
             return g
     return 1
+
+
+def measure_projection(wl, dev, d_model: int):
+    """Time lrkv_project_append (the fused latent projection + append that produces each
+    step's new latent rows) on this workload's cache shape, with a d_model-wide hidden
+    state. The factors A_K, A_V are rotated over >= 3x L2 of copies; every call appends
+    at a fresh slot. Returns a dict for the JSON line."""
+    g = torch.Generator(device="cpu").manual_seed(wl.seed + 99)
+    io_t = torch.float32 if wl.io_dtype == "f32" else torch.bfloat16
+    H, r, B = wl.n_kv_heads, wl.rank, wl.batch
+    a_bytes = 2 * H * d_model * r * (4 if wl.io_dtype == "f32" else 2)
+    n_a = max(2, min(48, math.ceil(3 * L2_BYTES / a_bytes)))
+    A = [(torch.randn(H, d_model, r, generator=g) / math.sqrt(d_model)).to(io_t).to(dev)
+         for _ in range(2 * n_a)]
+    x = torch.randn(B, d_model, generator=g).to(io_t).to(dev)
+    per_graph, replays, warm = 40, 3, 5
+    cap = warm + per_graph * (replays + 1) + 16
+    lat_t = {"f32": torch.float32, "bf16": torch.bfloat16, "i8": torch.int8,
+             "e4m3": torch.uint8}[wl.latent_dtype]
+    ZK = torch.zeros(B, H, cap, r, dtype=lat_t, device=dev)
+    ZV = torch.zeros_like(ZK)
+    quant = wl.latent_dtype in ("i8", "e4m3")
+    SK = torch.ones(B, H, cap, dtype=torch.float32, device=dev) if quant else None
+    SV = torch.ones_like(SK) if quant else None
+    seq = torch.zeros(B, dtype=torch.int32, device=dev)
+    dims = lrkv.make_dims(B, wl.n_q_heads, H, wl.d_head, r, cap, cap, wl.io_dtype,
+                          wl.latent_dtype)
+    ws = torch.zeros(max(lrkv.workspace_bytes(dims), 1 << 20), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    call = lambda i: lrkv.project_append(dims, x, A[2 * (i % n_a)], A[2 * (i % n_a) + 1], ZK, ZV,
+                                         SK, SV, seq, ws, stream=stream)
+    with torch.cuda.stream(stream):
+        for i in range(warm):
+            call(i)
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(per_graph):
+                call(i)
+        graph.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(replays):
+            graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    n = per_graph * replays
+    us = e0.elapsed_time(e1) * 1e3 / n
+    st = lrkv.read_status(ws)
+    if st:
+        raise RuntimeError(f"device status {st} after the projection timing")
+    lat_bytes = {"f32": 4, "bf16": 2, "i8": 1, "e4m3": 1}[wl.latent_dtype]
+    moved = a_bytes + x.numel() * x.element_size() + 2 * B * H * r * lat_bytes + (
+        2 * B * H * 4 if quant else 0)
+    peak, kind = peaks()
+    return {"d_model": d_model, "us_per_call": us, "bytes_per_call": moved,
+            "achieved_GBs": moved / (us * 1e-6) / 1e9, "peak_GBs": peak, "peak_kind": kind,
+            "frac": moved / (us * 1e-6) / 1e9 / peak, "launches": "CUDA graph of 40 calls",
+            "factors": f"rotated over {n_a} copies ({n_a * a_bytes / 1e6:.0f} MB)"}
 
 
 def run_ours(args, rank, world, local):
@@ -440,6 +507,8 @@ def run_ours(args, rank, world, local):
         "clocks": clocks,
         "cpu_baseline": None,
     }
+    if args.projection_dmodel > 0:
+        line["project_append"] = measure_projection(wl, dev, args.projection_dmodel)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         per_unit, n, lb, spent = oracle_sample(wl, inputs, args.cpu_seconds)
         cores = blas_threads()

@@ -208,7 +208,11 @@ int lrkv_decode_step_host(const lrkv_dims* dims, const void* q_host, const void*
  * int8 / e4m3 codes with a per-row fp32 absmax scale), then seqlens[b] += 1.
  *   x      [B][d_model], io dtype, device
  *   AK, AV [H_kv][d_model][rank], io dtype, device
- *   other arguments as lrkv_append (workspace: its header, >= 256 bytes).
+ *   other arguments as lrkv_append. The workspace needs its 256-byte header; the
+ *   bytes after it, when there are enough (a decode workspace of the same dims
+ *   usually has), hold partial sums so the hidden size is split over more CTAs.
+ *   The sums are added in a fixed order, so a call is deterministic for a given
+ *   workspace size (different sizes may split differently and round differently).
  * Errors: LRKV_ERR_DIMS (dims, d_model outside [1, 2^20]), LRKV_ERR_ARG (NULL pointer,
  * scales present iff quantised latents), LRKV_ERR_ALIGN, LRKV_ERR_WORKSPACE,
  * LRKV_ERR_LAUNCH. A row whose slot is past the capacity is left untouched, keeps its

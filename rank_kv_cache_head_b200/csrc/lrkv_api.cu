@@ -358,6 +358,8 @@ int lrkv_project_append(const lrkv_dims* dims, int32_t d_model, const void* x, c
   a.AK = AK;
   a.AV = AV;
   a.d_model = d_model;
+  a.nsplit = project_nsplit(a.app.Hkv, a.app.B, a.app.r, d_model, workspace_bytes);
+  a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + kHeaderBytes);
   if (launch_project_append(a, (cudaStream_t)stream) != cudaSuccess) return LRKV_ERR_LAUNCH;
   return LRKV_OK;
 }

@@ -80,6 +80,8 @@ struct ProjArgs {
   const void* AK;   // [Hkv][d_model][r], io dtype
   const void* AV;
   int d_model;
+  int nsplit;       // CTAs sharing one (KV head, K|V) over the hidden size
+  float* part;      // nsplit > 1: [2 Hkv][nsplit][B][r] partial sums (workspace)
 };
 
 // Programmatic dependent launch: every kernel of the library is launched so that it
@@ -115,6 +117,8 @@ cudaError_t launch_split_simt(const SplitArgs& a, const Plan& p, cudaStream_t st
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t st);
 cudaError_t launch_project_append(const ProjArgs& a, cudaStream_t st);
+// hidden-size split of the projection for this workspace size (1: none)
+int project_nsplit(int Hkv, int B, int r, int d_model, size_t workspace_bytes);
 
 // tcgen05 path: whether it supports these dims, its shared memory per CTA and CTAs
 // per SM, and the launcher.

@@ -338,12 +338,33 @@ __global__ void __launch_bounds__(1024) lrkv_append_kernel(AppendArgs a) {
 // is the token's hidden state times the down factor), accumulated in fp32 and
 // written at slot seqlens[b] exactly as lrkv_append writes a row (bf16 RNE, or int8 /
 // e4m3 codes with a per-row absmax scale). The last CTA to finish advances seqlens.
-// grid (2 Hkv): CTA = (KV head, K | V); 256 threads = column k (t % r) x row group
-// (t / r). It reads its factor once per group of 16 batch rows (later groups from
-// L2), with the rows of x staged in shared memory 256 columns at a time.
+// grid (2 Hkv, nsplit): CTA = (KV head, K | V, slice of the hidden size); 256 threads
+// = column k (t % r) x row group (t / r). Rows of x are staged in shared memory 256
+// columns at a time, 16 batch rows per pass. With nsplit > 1 every CTA writes its
+// partial sums to the workspace and the last CTA of a KV head adds them in a fixed
+// order and writes that head's rows (deterministic).
 constexpr int kProjThreads = 256;
 constexpr int kProjRows = 16;     // batch rows per pass (accumulators a thread)
 constexpr int kProjChunk = 256;   // columns of x staged per step
+constexpr int kProjMaxHeads = 60; // per-head counters live in header words 4..63
+
+template <int LAT>
+__device__ __forceinline__ void proj_write_rows(const ProjArgs& pa, int row, int b0, int nb,
+                                                const float* zs, int lane, int warp) {
+  const AppendArgs& a = pa.app;
+  for (int bb = warp; bb < nb; bb += kProjThreads / 32) {
+    const int b = b0 + bb;
+    const int slot = a.seqlens[b];
+    if (slot < 0 || slot >= a.Lcap) {
+      if (lane == 0) atomicOr(a.header + kStatusWord, LRKV_STATUS_APPEND_FULL);
+      continue;
+    }
+    float zz[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) zz[e] = (lane + 32 * e < a.r) ? zs[bb * a.r + lane + 32 * e] : 0.f;
+    append_row<LAT>(a, b, row, slot, lane, zz);
+  }
+}
 
 template <int LAT>
 __global__ void __launch_bounds__(kProjThreads) lrkv_project_append_kernel(ProjArgs pa) {
@@ -353,12 +374,14 @@ __global__ void __launch_bounds__(kProjThreads) lrkv_project_append_kernel(ProjA
   griddep_wait();
   griddep_launch_dependents();
   const AppendArgs& a = pa.app;
-  const int g = blockIdx.x >> 1, kv = blockIdx.x & 1;
+  const int gk = blockIdx.x, g = gk >> 1, kv = gk & 1, sp = blockIdx.y, ns = pa.nsplit;
   const int r = a.r, t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int ngr = kProjThreads / r;                 // row groups (r divides into 256 or not)
+  const int ngr = kProjThreads / r;                 // row groups
   const int k = t % r, rg = t / r;
   const bool active = rg < ngr;
   const int D = pa.d_model;
+  const int dspan = ((D + ns - 1) / ns + kProjChunk - 1) / kProjChunk * kProjChunk;
+  const int dlo = min(D, sp * dspan), dhi = min(D, dlo + dspan);
   const void* A = kv ? pa.AV : pa.AK;
   const size_t abase = (size_t)g * D * r;
   for (int b0 = 0; b0 < a.B; b0 += kProjRows) {
@@ -366,16 +389,28 @@ __global__ void __launch_bounds__(kProjThreads) lrkv_project_append_kernel(ProjA
     float acc[kProjRows];
 #pragma unroll
     for (int bb = 0; bb < kProjRows; ++bb) acc[bb] = 0.f;
-    for (int d0 = 0; d0 < D; d0 += kProjChunk) {
+    for (int d0 = dlo; d0 < dhi; d0 += kProjChunk) {
       __syncthreads();
       for (int idx = t; idx < kProjRows * kProjChunk; idx += kProjThreads) {
         const int bb = idx / kProjChunk, dd = idx - bb * kProjChunk;
-        xs[idx] = (bb < nb && d0 + dd < D) ? load_io(pa.x, (size_t)(b0 + bb) * D + d0 + dd, a.io_dtype) : 0.f;
+        xs[idx] = (bb < nb && d0 + dd < dhi) ? load_io(pa.x, (size_t)(b0 + bb) * D + d0 + dd, a.io_dtype) : 0.f;
       }
       __syncthreads();
       if (active) {
-        const int dn = min(kProjChunk, D - d0);
-        for (int i = rg; i < dn; i += ngr) {
+        const int dn = min(kProjChunk, dhi - d0);
+        int i = rg;
+        // eight rows of the factor in flight a thread (the loop is load-latency-bound)
+        for (; i + 7 * ngr < dn; i += 8 * ngr) {
+          float av[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) av[u] = load_io(A, abase + (size_t)(d0 + i + u * ngr) * r + k, a.io_dtype);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+#pragma unroll
+            for (int bb = 0; bb < kProjRows; ++bb)
+              acc[bb] = fmaf(xs[bb * kProjChunk + i + u * ngr], av[u], acc[bb]);
+        }
+        for (; i < dn; i += ngr) {
           const float av = load_io(A, abase + (size_t)(d0 + i) * r + k, a.io_dtype);
 #pragma unroll
           for (int bb = 0; bb < kProjRows; ++bb) acc[bb] = fmaf(xs[bb * kProjChunk + i], av, acc[bb]);
@@ -393,29 +428,47 @@ __global__ void __launch_bounds__(kProjThreads) lrkv_project_append_kernel(ProjA
       const int bb = idx / r, kk = idx - bb * r;
       float z = 0.f;
       for (int q = 0; q < ngr; ++q) z += red[(q * kProjRows + bb) * r + kk];
-      zs[bb * r + kk] = z;
+      if (ns == 1) zs[bb * r + kk] = z;
+      else pa.part[(((size_t)gk * ns + sp) * a.B + b0 + bb) * r + kk] = z;
     }
     __syncthreads();
-    // one warp per batch row writes the row (and its scale) at the row's slot
-    for (int bb = warp; bb < nb; bb += kProjThreads / 32) {
-      const int b = b0 + bb;
-      const int slot = a.seqlens[b];
-      if (slot < 0 || slot >= a.Lcap) {
-        if (lane == 0) atomicOr(a.header + kStatusWord, LRKV_STATUS_APPEND_FULL);
-        continue;
-      }
-      float zz[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) zz[e] = (lane + 32 * e < r) ? zs[bb * r + lane + 32 * e] : 0.f;
-      append_row<LAT>(a, b, 2 * g + kv, slot, lane, zz);
-    }
+    if (ns == 1) proj_write_rows<LAT>(pa, 2 * g + kv, b0, nb, zs, lane, warp);
   }
-  // the last CTA to finish advances every valid row's length (all CTAs have read it)
+  if (ns > 1) {
+    // the last of the head's 2 nsplit CTAs adds the slices (fixed order) and writes
+    // the head's K and V rows
+    __syncthreads();
+    bool last = false;
+    if (t == 0) {
+      __threadfence();
+      last = atomicAdd(a.header + 4 + g, 1u) == 2u * ns - 1u;
+    }
+    if (!__syncthreads_or(last)) return;
+    __threadfence();
+    for (int kvv = 0; kvv < 2; ++kvv) {
+      for (int b0 = 0; b0 < a.B; b0 += kProjRows) {
+        const int nb = min(kProjRows, a.B - b0);
+        __syncthreads();
+        for (int idx = t; idx < nb * r; idx += kProjThreads) {
+          const int bb = idx / r, kk = idx - bb * r;
+          float z = 0.f;
+          for (int q = 0; q < ns; ++q)
+            z += __ldcg(&pa.part[((((size_t)(2 * g + kvv)) * ns + q) * a.B + b0 + bb) * r + kk]);
+          zs[bb * r + kk] = z;
+        }
+        __syncthreads();
+        proj_write_rows<LAT>(pa, 2 * g + kvv, b0, nb, zs, lane, warp);
+      }
+    }
+    if (t == 0) atomicExch(a.header + 4 + g, 0u);
+  }
+  // the last writer advances every valid row's length (all writers have read it)
   __syncthreads();
   if (t == 0) {
     __threadfence();
+    const unsigned writers = ns > 1 ? (unsigned)a.Hkv : gridDim.x;
     const unsigned prev = atomicAdd(a.header + kProjCounter, 1u);
-    if (prev == gridDim.x - 1) {
+    if (prev == writers - 1) {
       __threadfence();
       for (int b = 0; b < a.B; ++b) {
         const int slot = a.seqlens[b];
@@ -470,13 +523,23 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_project_append(const ProjArgs& a, cudaStream_t st) {
-  const dim3 grid(2 * a.app.Hkv), block(kProjThreads);
+  const dim3 grid(2 * a.app.Hkv, a.nsplit), block(kProjThreads);
   switch (a.app.latent_dtype) {
     case LRKV_F32: return launch_pdl(lrkv_project_append_kernel<LRKV_F32>, grid, block, 0, st, a);
     case LRKV_BF16: return launch_pdl(lrkv_project_append_kernel<LRKV_BF16>, grid, block, 0, st, a);
     case LRKV_I8: return launch_pdl(lrkv_project_append_kernel<LRKV_I8>, grid, block, 0, st, a);
     default: return launch_pdl(lrkv_project_append_kernel<LRKV_E4M3>, grid, block, 0, st, a);
   }
+}
+
+int project_nsplit(int Hkv, int B, int r, int d_model, size_t workspace_bytes) {
+  if (Hkv > kProjMaxHeads) return 1;
+  int ns = (2 * num_sms() + 2 * Hkv - 1) / (2 * Hkv);
+  ns = std::min(ns, std::max(1, d_model / kProjChunk));
+  const size_t per = (size_t)2 * Hkv * B * r * sizeof(float);
+  const size_t room = workspace_bytes > kHeaderBytes ? workspace_bytes - kHeaderBytes : 0;
+  ns = (int)std::min<size_t>((size_t)ns, room / per);
+  return std::max(1, ns);
 }
 
 }  // namespace lrkv

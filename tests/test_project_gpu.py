@@ -24,10 +24,11 @@ def _decode(bits, lat):
     return orc.decode_stored(bits, lat)
 
 
+@pytest.mark.parametrize("ws_bytes", [256, 4 << 20])   # header only: no split; room: split
 @pytest.mark.parametrize("io,lat,r,D", [("f32", "f32", 32, 300), ("bf16", "bf16", 32, 300),
                                         ("bf16", "bf16", 48, 1000), ("bf16", "i8", 32, 520),
-                                        ("bf16", "e4m3", 64, 256)])
-def test_project_append_matches_oracle(io, lat, r, D):
+                                        ("bf16", "e4m3", 64, 2304)])
+def test_project_append_matches_oracle(io, lat, r, D, ws_bytes):
     B, H, Lcap = 3, 2, 64
     rng = np.random.default_rng(1000 + r + D)
     x = torch.from_numpy(rng.standard_normal((B, D))).to(_IO[io])
@@ -49,7 +50,7 @@ def test_project_append_matches_oracle(io, lat, r, D):
     SK = None if S0 is None else S0[0].clone().cuda()
     SV = None if S0 is None else S0[1].clone().cuda()
     seq = seq0.clone().cuda()
-    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
     lrkv.project_append(dims, x.cuda(), AK.cuda(), AV.cuda(), ZK, ZV, SK, SV, seq, ws)
     status = lrkv.read_status(ws)
     assert status & lrkv.STATUS_APPEND_FULL
