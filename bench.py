@@ -479,6 +479,9 @@ def run_ours(args, rank, world, local):
     split_mean_ms = statistics.mean(split_ms)
     achieved = sb["split_kernel"] / (split_mean_ms * 1e-3) / 1e9
     traffic = profiled_traffic(args.workload, plan["algo"])
+    if plan.get("device_chunk"):
+        # the split size the kernel picked from the lengths (header word 4)
+        plan["chunk_chosen"] = int(ws[16:20].view(torch.int32).item())
     e2e_value = sum_over_ranks(e2e_lat, dev) / (e2e_ms * 1e-3) / 1e9
     io_bytes = 4 if wl.io_dtype == "f32" else 2
     line = {

@@ -114,11 +114,15 @@ typedef struct {
 /* What lrkv_decode_attn will do for these dims (for tests and benchmarks). */
 typedef struct {
   int32_t algo;         /* LRKV_ALGO_SIMT or LRKV_ALGO_TCGEN05 */
-  int32_t num_splits;   /* S: splits per (batch row, KV head) at max_seqlen */
-  int32_t chunk;        /* tokens per split (a multiple of 128) */
+  int32_t num_splits;   /* S: the most splits per (batch row, KV head), at max_seqlen */
+  int32_t chunk;        /* tokens per split (a multiple of 128); with device_chunk the
+                           finest the kernel may pick */
   int32_t grid;         /* CTAs of the split kernel */
   int32_t smem_bytes;   /* dynamic shared memory of the split kernel */
-  int32_t reserved[3];
+  int32_t full_chunk;   /* tokens per split when every row is at max_seqlen */
+  int32_t device_chunk; /* 1: the kernel scales full_chunk by the share of 128-token
+                           tiles the rows hold (clamped to [chunk, full_chunk]) */
+  int32_t reserved;
 } lrkv_plan_info;
 
 /* Fill *plan for dims. Returns 0 or a negative code. */
@@ -207,7 +211,7 @@ int lrkv_decode_step_host(const lrkv_dims* dims, const void* q_host, const void*
  * written at slot seqlens[b] exactly as lrkv_append writes a row (fp32, bf16 RNE, or
  * int8 / e4m3 codes with a per-row fp32 absmax scale), then seqlens[b] += 1.
  *   x      [B][d_model], io dtype, device
- *   AK, AV [H_kv][d_model][rank], io dtype, device
+ *   AK, AV [H_kv][d_model][rank], io dtype, device, 16-byte aligned
  *   other arguments as lrkv_append. The workspace needs its 256-byte header; the
  *   bytes after it, when there are enough (a decode workspace of the same dims
  *   usually has), hold partial sums so the hidden size is split over more CTAs.
@@ -216,7 +220,8 @@ int lrkv_decode_step_host(const lrkv_dims* dims, const void* q_host, const void*
  * Errors: LRKV_ERR_DIMS (dims, d_model outside [1, 2^20]), LRKV_ERR_ARG (NULL pointer,
  * scales present iff quantised latents), LRKV_ERR_ALIGN, LRKV_ERR_WORKSPACE,
  * LRKV_ERR_LAUNCH. A row whose slot is past the capacity is left untouched, keeps its
- * length and sets LRKV_STATUS_APPEND_FULL.
+ * length and sets LRKV_STATUS_APPEND_FULL. LRKV_STATUS_TIMEOUT: the wait for a factor
+ * copy into shared memory ran out after one second (the appended rows are invalid).
  */
 int lrkv_project_append(const lrkv_dims* dims, int32_t d_model, const void* x, const void* AK,
                         const void* AV, void* ZK, void* ZV, float* ZK_scale, float* ZV_scale,

@@ -132,6 +132,14 @@ int make_plan(const lrkv_dims* d, Plan* p) {
       memo[key] = chunk_tiles;
     }
   }
+  p->device_chunk = 0;
+  p->chunk_hint = chunk_tiles;
+  if (p->algo == LRKV_ALGO_TCGEN05 && d->num_splits == 0 && chunk_tiles > 1) {
+    // the kernel scales the split size down to the tiles the rows actually hold;
+    // the plan (workspace, merge bound) is for the finest it may pick
+    p->device_chunk = 1;
+    chunk_tiles = (chunk_tiles + 3) / 4;
+  }
   p->S = (tiles_max + chunk_tiles - 1) / chunk_tiles;
   p->chunk = chunk_tiles * kTile;
   if (p->algo == LRKV_ALGO_TCGEN05) {
@@ -184,6 +192,8 @@ int lrkv_plan(const lrkv_dims* dims, lrkv_plan_info* info) {
   info->chunk = p.chunk;
   info->grid = p.grid;
   info->smem_bytes = p.smem;
+  info->full_chunk = p.chunk_hint * kTile;
+  info->device_chunk = p.device_chunk;
   return LRKV_OK;
 }
 
@@ -265,6 +275,8 @@ int lrkv_decode_attn_timed(const lrkv_dims* dims, const void* q, const void* ZK,
   a.latent_dtype = dims->latent_dtype;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_head));
   a.debug_stall = 0;
+  a.device_chunk = 0;
+  a.chunk_hint = p.chunk_hint;
 
   if (p.algo == LRKV_ALGO_TCGEN05 && quant &&
       ((reinterpret_cast<uintptr_t>(ZK_scale) | reinterpret_cast<uintptr_t>(ZV_scale)) & 15u)) {
@@ -273,7 +285,10 @@ int lrkv_decode_attn_timed(const lrkv_dims* dims, const void* q, const void* ZK,
     p.smem = (int)simt_smem_bytes(dims->rank, dims->d_head, dims->n_q_heads / dims->n_kv_heads);
     if (p.smem > 227 * 1024) return LRKV_ERR_UNSUPPORTED;
   }
-  if (p.algo == LRKV_ALGO_TCGEN05) a.debug_stall = g_debug_stall.exchange(0);
+  if (p.algo == LRKV_ALGO_TCGEN05) {
+    a.debug_stall = g_debug_stall.exchange(0);
+    a.device_chunk = p.device_chunk;
+  }
   record_event(ev_split_begin, st);
   cudaError_t e = (p.algo == LRKV_ALGO_TCGEN05) ? launch_split_tc(a, p, st)
                                                 : launch_split_simt(a, p, st);
@@ -295,6 +310,7 @@ int lrkv_decode_attn_timed(const lrkv_dims* dims, const void* q, const void* ZK,
   m.Lcap = a.Lcap;
   m.max_seqlen = a.max_seqlen;
   m.io_dtype = a.io_dtype;
+  m.device_chunk = a.device_chunk;
   if (launch_merge(m, st) != cudaSuccess) return LRKV_ERR_LAUNCH;
   return LRKV_OK;
 }
@@ -338,7 +354,9 @@ int lrkv_project_append(const lrkv_dims* dims, int32_t d_model, const void* x, c
   if (!x || !AK || !AV || !ZK || !ZV || !seqlens || !workspace) return LRKV_ERR_ARG;
   if (quant != (ZK_scale != nullptr) || quant != (ZV_scale != nullptr)) return LRKV_ERR_ARG;
   if (workspace_bytes < kHeaderBytes) return LRKV_ERR_WORKSPACE;
-  if (!aligned16(ZK) || !aligned16(ZV) || !aligned16(workspace)) return LRKV_ERR_ALIGN;
+  if (!aligned16(ZK) || !aligned16(ZV) || !aligned16(workspace) || !aligned16(AK) ||
+      !aligned16(AV))
+    return LRKV_ERR_ALIGN;
   ProjArgs a;
   a.app.zk_new = nullptr;
   a.app.zv_new = nullptr;
@@ -358,7 +376,8 @@ int lrkv_project_append(const lrkv_dims* dims, int32_t d_model, const void* x, c
   a.AK = AK;
   a.AV = AV;
   a.d_model = d_model;
-  a.nsplit = project_nsplit(a.app.Hkv, a.app.B, a.app.r, d_model, workspace_bytes);
+  a.nsplit = project_nsplit(a.app.Hkv, a.app.B, a.app.r, d_model,
+                            (int)dtype_bytes(dims->io_dtype), workspace_bytes);
   a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + kHeaderBytes);
   if (launch_project_append(a, (cudaStream_t)stream) != cudaSuccess) return LRKV_ERR_LAUNCH;
   return LRKV_OK;

@@ -15,13 +15,19 @@ constexpr int kTile = 128;            // tokens per pipeline tile / split granul
 constexpr size_t kHeaderBytes = 256;  // workspace header: status word + counters
 
 // Workspace header words.
-enum HeaderWord { kStatusWord = 0, kWorkCounter = 1, kDoneCounter = 2, kProjCounter = 3 };
+enum HeaderWord {
+  kStatusWord = 0, kWorkCounter = 1, kDoneCounter = 2, kProjCounter = 3,
+  kChunkWord = 4,      // split size chosen on the device (tokens), read by the merge
+  kProjHeadWord = 8,   // words 8..63: per-KV-head counters of the projection
+};
 
 // Launch plan for one call (depends only on dims and the device).
 struct Plan {
   int algo;         // LRKV_ALGO_SIMT or LRKV_ALGO_TCGEN05
   int S;            // splits per (b, KV head) at max_seqlen
-  int chunk;        // tokens per split, multiple of kTile
+  int chunk;        // tokens per split, multiple of kTile (device_chunk: the finest)
+  int device_chunk; // the tensor-core kernel picks the split size from the actual lengths
+  int chunk_hint;   // device_chunk: tiles per split for rows at full length
   int grid;         // CTAs of the split kernel
   int smem;         // dynamic shared memory of the split kernel
   size_t lse_off;   // byte offset of lse partials in the workspace
@@ -46,6 +52,8 @@ struct SplitArgs {
   int io_dtype, latent_dtype;
   float scale_log2;  // log2(e) / sqrt(d)
   int debug_stall;   // test hook: work unit 0's first tile is withheld (see lrkv.h)
+  int device_chunk;  // choose the split size on the device (chunk = the finest, S its bound)
+  int chunk_hint;    // device_chunk: the split size, in tiles, for rows at full length
 };
 
 struct MergeArgs {
@@ -57,6 +65,7 @@ struct MergeArgs {
   uint32_t* header;
   int B, Hq, d, S, chunk, Lcap, max_seqlen;
   int io_dtype;
+  int device_chunk;  // read the split size the split kernel chose from the header
 };
 
 struct AppendArgs {
@@ -118,7 +127,7 @@ cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t st);
 cudaError_t launch_project_append(const ProjArgs& a, cudaStream_t st);
 // hidden-size split of the projection for this workspace size (1: none)
-int project_nsplit(int Hkv, int B, int r, int d_model, size_t workspace_bytes);
+int project_nsplit(int Hkv, int B, int r, int d_model, int io_bytes, size_t workspace_bytes);
 
 // tcgen05 path: whether it supports these dims, its shared memory per CTA and CTAs
 // per SM, and the launcher.

@@ -16,9 +16,12 @@
 #include <math_constants.h>
 
 #include "lrkv_internal.h"
+#include "lrkv_sm100.cuh"
 
 namespace lrkv {
 namespace {
+
+using namespace sm100;
 
 constexpr int kSimtThreads = 256;
 constexpr int kSimtTile = 32;  // tokens per inner tile of the CUDA-core kernel
@@ -211,7 +214,10 @@ __global__ void __launch_bounds__(128) lrkv_merge(MergeArgs a) {
   for (int k = 0; k < kPre; ++k) opre[k] = (active && k < a.S) ? o[(size_t)k * a.d + tid] : 0.f;
   const int L = checked_len(a.seqlens, b, a.Lcap, a.max_seqlen, a.header,
                             (bh % a.Hq) == 0 && tid == 0);
-  const int ns = min(a.S, (L + a.chunk - 1) / a.chunk);
+  // the split size: the plan's, or the one the tensor-core split kernel chose
+  const int chunk = a.device_chunk ? (int)*reinterpret_cast<volatile uint32_t*>(a.header + kChunkWord)
+                                   : a.chunk;
+  const int ns = min(a.S, (L + chunk - 1) / chunk);
   if (tid < 32) {
     float mx = lane < ns ? lse0 : -CUDART_INF_F;
     for (int s = lane + 32; s < ns; s += 32) mx = fmaxf(mx, lse[s]);
@@ -338,21 +344,44 @@ __global__ void __launch_bounds__(1024) lrkv_append_kernel(AppendArgs a) {
 // is the token's hidden state times the down factor), accumulated in fp32 and
 // written at slot seqlens[b] exactly as lrkv_append writes a row (bf16 RNE, or int8 /
 // e4m3 codes with a per-row absmax scale). The last CTA to finish advances seqlens.
-// grid (2 Hkv, nsplit): CTA = (KV head, K | V, slice of the hidden size); 256 threads
-// = column k (t % r) x row group (t / r). Rows of x are staged in shared memory 256
-// columns at a time, 16 batch rows per pass. With nsplit > 1 every CTA writes its
-// partial sums to the workspace and the last CTA of a KV head adds them in a fixed
-// order and writes that head's rows (deterministic).
+// grid (2 Hkv, nsplit): CTA = (KV head, K | V, slice of the hidden size), 256
+// threads. One thread issues a bulk copy of the CTA's factor rows into shared memory
+// (they are contiguous in A) while the others stage rows of x as fp32, so the factor
+// crosses HBM once and every later pass over the batch reads it from shared memory.
+// A factor row (r columns) is read by tpr lanes, 8 columns each (tpr = r / 8 rounded up
+// to a power of two); the other lanes of the warp and the 8 warps take other rows.
+// Each thread keeps 8 batch rows x 8 columns of fp32 sums in packed pairs
+// (fma.rn.f32x2). The sums are reduced over the lanes that share columns (a butterfly
+// in which each step halves the values a lane holds), then over the warps in a fixed
+// order. With nsplit > 1 every CTA writes its partial sums to the workspace and the
+// last CTA of a KV head adds them in a fixed order and writes that head's rows
+// (deterministic). A slice larger than the shared-memory budget is taken in chunks,
+// copied again for every pass.
 constexpr int kProjThreads = 256;
-constexpr int kProjRows = 16;     // batch rows per pass (accumulators a thread)
-constexpr int kProjChunk = 256;   // columns of x staged per step
-constexpr int kProjMaxHeads = 60; // per-head counters live in header words 4..63
+constexpr int kProjWarps = kProjThreads / 32;
+constexpr int kProjRows = 8;              // batch rows per pass
+constexpr int kProjMaxChunk = 1024;       // factor rows staged at a time, at most
+constexpr int kProjABytes = 64 * 1024;    // shared-memory budget for factor rows
+constexpr int kProjMinSpan = 64;          // fewest hidden-size rows a CTA takes when splitting
+constexpr int kProjMaxHeads = 56;         // per-head counters live in header words 8..63
+
+// factor rows a CTA stages at a time, for row width r and element size e
+__host__ __device__ inline int proj_chunk_rows(int r, int e, int dspan) {
+  const int cap = min(kProjMaxChunk, kProjABytes / (r * e));
+  return max(1, min(cap, dspan));
+}
+
+// dynamic shared memory: barrier, factor rows, x rows (or the warps' partial sums), sums
+__host__ __device__ inline size_t proj_smem_bytes(int r, int e, int cr) {
+  const size_t xs = (size_t)kProjRows * cr, red = (size_t)kProjWarps * kProjRows * r;
+  return 16 + (size_t)cr * r * e + sizeof(float) * ((xs > red ? xs : red) + (size_t)kProjRows * r);
+}
 
 template <int LAT>
 __device__ __forceinline__ void proj_write_rows(const ProjArgs& pa, int row, int b0, int nb,
                                                 const float* zs, int lane, int warp) {
   const AppendArgs& a = pa.app;
-  for (int bb = warp; bb < nb; bb += kProjThreads / 32) {
+  for (int bb = warp; bb < nb; bb += kProjWarps) {
     const int b = b0 + bb;
     const int slot = a.seqlens[b];
     if (slot < 0 || slot >= a.Lcap) {
@@ -366,73 +395,160 @@ __device__ __forceinline__ void proj_write_rows(const ProjArgs& pa, int row, int
   }
 }
 
-template <int LAT>
-__global__ void __launch_bounds__(kProjThreads) lrkv_project_append_kernel(ProjArgs pa) {
-  __shared__ float xs[kProjRows * kProjChunk];
-  __shared__ float red[kProjThreads * kProjRows];   // [row group][batch row][column]
-  __shared__ float zs[kProjRows * 256];
+// 8 consecutive factor columns as 4 packed fp32 pairs, from shared memory
+template <int IO>
+__device__ __forceinline__ void proj_row8(const char* p, uint64_t (&a2)[4]) {
+  if constexpr (IO == LRKV_F32) {
+    const uint4 w0 = reinterpret_cast<const uint4*>(p)[0];
+    const uint4 w1 = reinterpret_cast<const uint4*>(p)[1];
+    a2[0] = pack2(__uint_as_float(w0.x), __uint_as_float(w0.y));
+    a2[1] = pack2(__uint_as_float(w0.z), __uint_as_float(w0.w));
+    a2[2] = pack2(__uint_as_float(w1.x), __uint_as_float(w1.y));
+    a2[3] = pack2(__uint_as_float(w1.z), __uint_as_float(w1.w));
+  } else {
+    const uint4 w = *reinterpret_cast<const uint4*>(p);
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j)   // bf16 -> fp32 is exact: the bits move up
+      a2[j] = pack2(__uint_as_float(u[j] << 16), __uint_as_float(u[j] & 0xffff0000u));
+  }
+}
+
+template <int LAT, int IO>
+__global__ void __launch_bounds__(kProjThreads, 2) lrkv_project_append_kernel(ProjArgs pa) {
+  constexpr int E = IO == LRKV_F32 ? 4 : 2;          // bytes an element
+  constexpr uint64_t kWaitNs = 1000000000ull;        // bounded waits: one second
+  extern __shared__ __align__(16) unsigned char proj_smem[];
+  __shared__ int abort_flag;
+  const AppendArgs& a = pa.app;
+  const int r = a.r;
+  const int gk = blockIdx.x, g = gk >> 1, kv = gk & 1, sp = blockIdx.y, ns = pa.nsplit;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int D = pa.d_model;
+  const int dspan = (D + ns - 1) / ns;
+  const int dlo = min(D, sp * dspan), dhi = min(D, dlo + dspan);
+  const int cr = proj_chunk_rows(r, E, dspan);
+  const int nchunks = max(1, (dhi - dlo + cr - 1) / cr);
+  const bool resident = nchunks == 1;
+  const uint32_t bar = smem_addr(proj_smem);
+  char* As = reinterpret_cast<char*>(proj_smem + 16);              // [row][r] as in A
+  float* xs = reinterpret_cast<float*>(As + (size_t)cr * r * E);   // [batch row][row]
+  float* red = xs;                                                 // [warp][batch row][col]
+  const size_t xs_floats = (size_t)kProjRows * cr, red_floats = (size_t)kProjWarps * kProjRows * r;
+  float* zs = xs + (xs_floats > red_floats ? xs_floats : red_floats);   // [batch row][col]
+  const char* A = static_cast<const char*>(kv ? pa.AV : pa.AK) + (size_t)g * D * r * E;
+  const size_t row_bytes = (size_t)r * E;
+  if (t == 0) {
+    abort_flag = 0;
+    mbar_init(bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
   griddep_wait();
   griddep_launch_dependents();
-  const AppendArgs& a = pa.app;
-  const int gk = blockIdx.x, g = gk >> 1, kv = gk & 1, sp = blockIdx.y, ns = pa.nsplit;
-  const int r = a.r, t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int ngr = kProjThreads / r;                 // row groups
-  const int k = t % r, rg = t / r;
-  const bool active = rg < ngr;
-  const int D = pa.d_model;
-  const int dspan = ((D + ns - 1) / ns + kProjChunk - 1) / kProjChunk * kProjChunk;
-  const int dlo = min(D, sp * dspan), dhi = min(D, dlo + dspan);
-  const void* A = kv ? pa.AV : pa.AK;
-  const size_t abase = (size_t)g * D * r;
+  uint32_t copies = 0;     // bulk copies issued so far (the barrier's phase count)
+  bool timed_out = false;
+  auto issue = [&](int d0, int dn) {
+    if (t == 0 && dn > 0) {
+      mbar_arrive_expect_tx(bar, (uint32_t)(dn * row_bytes));
+      bulk_load(smem_addr(As), A + (size_t)d0 * row_bytes, (uint32_t)(dn * row_bytes), bar);
+    }
+    if (dn > 0) ++copies;
+  };
+  if (resident) issue(dlo, dhi - dlo);
+
+  int tpr = 1;
+  while (tpr * 8 < r) tpr <<= 1;
+  const int spw = 32 / tpr, c0 = (lane & (tpr - 1)) * 8;
+  const int nslots = kProjWarps * spw, slot = warp * spw + lane / tpr;
+  const bool active = c0 < r;
+
   for (int b0 = 0; b0 < a.B; b0 += kProjRows) {
     const int nb = min(kProjRows, a.B - b0);
-    float acc[kProjRows];
+    uint64_t acc[kProjRows][4];
 #pragma unroll
-    for (int bb = 0; bb < kProjRows; ++bb) acc[bb] = 0.f;
-    for (int d0 = dlo; d0 < dhi; d0 += kProjChunk) {
+    for (int bb = 0; bb < kProjRows; ++bb)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[bb][j] = 0ull;
+    for (int ch = 0; ch < nchunks; ++ch) {
+      const int d0 = dlo + ch * cr, dn = min(cr, dhi - d0);
+      __syncthreads();                           // the previous chunk / pass is consumed
+      if (!resident) issue(d0, dn);
+      for (int bb = 0; bb < kProjRows; ++bb)
+        for (int i = t; i < cr; i += kProjThreads)
+          xs[bb * cr + i] = (bb < nb && i < dn) ? load_io(pa.x, (size_t)(b0 + bb) * D + d0 + i, IO) : 0.f;
       __syncthreads();
-      for (int idx = t; idx < kProjRows * kProjChunk; idx += kProjThreads) {
-        const int bb = idx / kProjChunk, dd = idx - bb * kProjChunk;
-        xs[idx] = (bb < nb && d0 + dd < dhi) ? load_io(pa.x, (size_t)(b0 + bb) * D + d0 + dd, a.io_dtype) : 0.f;
-      }
-      __syncthreads();
+      if (dn > 0 && !mbar_wait(bar, (copies - 1) & 1, &abort_flag, kWaitNs)) timed_out = true;
       if (active) {
-        const int dn = min(kProjChunk, dhi - d0);
-        int i = rg;
-        // eight rows of the factor in flight a thread (the loop is load-latency-bound)
-        for (; i + 7 * ngr < dn; i += 8 * ngr) {
-          float av[8];
+        for (int i = slot; i < dn; i += nslots) {
+          uint64_t a2[4];
+          proj_row8<IO>(As + (size_t)i * row_bytes + (size_t)c0 * E, a2);
 #pragma unroll
-          for (int u = 0; u < 8; ++u) av[u] = load_io(A, abase + (size_t)(d0 + i + u * ngr) * r + k, a.io_dtype);
+          for (int bb = 0; bb < kProjRows; ++bb) {
+            const float xv = xs[bb * cr + i];
+            const uint64_t x2 = pack2(xv, xv);
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-#pragma unroll
-            for (int bb = 0; bb < kProjRows; ++bb)
-              acc[bb] = fmaf(xs[bb * kProjChunk + i + u * ngr], av[u], acc[bb]);
-        }
-        for (; i < dn; i += ngr) {
-          const float av = load_io(A, abase + (size_t)(d0 + i) * r + k, a.io_dtype);
-#pragma unroll
-          for (int bb = 0; bb < kProjRows; ++bb) acc[bb] = fmaf(xs[bb * kProjChunk + i], av, acc[bb]);
+            for (int j = 0; j < 4; ++j) acc[bb][j] = ffma2p(x2, a2[j], acc[bb][j]);
+          }
         }
       }
     }
-    __syncthreads();
+    // lanes that share columns: each butterfly step sends half of the values a lane
+    // holds to its partner and keeps the other half, so after s steps a lane holds
+    // 64 / 2^s sums; which ones depends on the lane's bits (index base `off`)
+    float v[64];
+#pragma unroll
+    for (int bb = 0; bb < kProjRows; ++bb)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = unpack2(acc[bb][j]);
+        v[bb * 8 + 2 * j] = f.x;
+        v[bb * 8 + 2 * j + 1] = f.y;
+      }
+    int off = 0, held = 64;
+#pragma unroll
+    for (int s = 0; s < 5; ++s) {
+      const int h = 32 >> s;                     // values sent (and kept) in this step
+      const int o = tpr << s;
+      if (o < 32) {
+        const bool hi = lane & o;
+#pragma unroll
+        for (int j = 0; j < h; ++j) {
+          const float send = hi ? v[j] : v[j + h];
+          const float keep = hi ? v[j + h] : v[j];
+          v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+        if (hi) off += h;
+        held = h;
+      }
+    }
+    __syncthreads();                             // every thread is done with xs
     if (active) {
 #pragma unroll
-      for (int bb = 0; bb < kProjRows; ++bb) red[(rg * kProjRows + bb) * r + k] = acc[bb];
+      for (int j = 0; j < 64; ++j) {
+        if (j < held) {
+          const int idx = off + j, bb = idx >> 3, c = idx & 7;
+          red[(warp * kProjRows + bb) * r + c0 + c] = v[j];
+        }
+      }
     }
     __syncthreads();
-    // the row groups' partial sums in a fixed order
     for (int idx = t; idx < nb * r; idx += kProjThreads) {
-      const int bb = idx / r, kk = idx - bb * r;
+      const int bb = idx / r, k = idx - bb * r;
       float z = 0.f;
-      for (int q = 0; q < ngr; ++q) z += red[(q * kProjRows + bb) * r + kk];
-      if (ns == 1) zs[bb * r + kk] = z;
-      else pa.part[(((size_t)gk * ns + sp) * a.B + b0 + bb) * r + kk] = z;
+#pragma unroll
+      for (int w = 0; w < kProjWarps; ++w) z += red[(w * kProjRows + bb) * r + k];
+      if (ns == 1) zs[idx] = z;
+      else pa.part[(((size_t)gk * ns + sp) * a.B + b0) * r + idx] = z;
     }
     __syncthreads();
     if (ns == 1) proj_write_rows<LAT>(pa, 2 * g + kv, b0, nb, zs, lane, warp);
+  }
+  if (timed_out) {
+    // results are invalid; make sure no copy still writes this CTA's shared memory
+    if (t == 0) atomicOr(a.header + kStatusWord, LRKV_STATUS_TIMEOUT);
+    abort_flag = 0;
+    mbar_wait(bar, (copies - 1) & 1, &abort_flag, kWaitNs);
   }
   if (ns > 1) {
     // the last of the head's 2 nsplit CTAs adds the slices (fixed order) and writes
@@ -441,7 +557,7 @@ __global__ void __launch_bounds__(kProjThreads) lrkv_project_append_kernel(ProjA
     bool last = false;
     if (t == 0) {
       __threadfence();
-      last = atomicAdd(a.header + 4 + g, 1u) == 2u * ns - 1u;
+      last = atomicAdd(a.header + kProjHeadWord + g, 1u) == 2u * ns - 1u;
     }
     if (!__syncthreads_or(last)) return;
     __threadfence();
@@ -460,7 +576,7 @@ __global__ void __launch_bounds__(kProjThreads) lrkv_project_append_kernel(ProjA
         proj_write_rows<LAT>(pa, 2 * g + kvv, b0, nb, zs, lane, warp);
       }
     }
-    if (t == 0) atomicExch(a.header + 4 + g, 0u);
+    if (t == 0) atomicExch(a.header + kProjHeadWord + g, 0u);
   }
   // the last writer advances every valid row's length (all writers have read it)
   __syncthreads();
@@ -522,20 +638,44 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t st) {
   }
 }
 
+template <int LAT, int IO>
+cudaError_t launch_project_typed(const ProjArgs& a, cudaStream_t st) {
+  const int e = IO == LRKV_F32 ? 4 : 2;
+  const int dspan = (a.d_model + a.nsplit - 1) / a.nsplit;
+  const size_t smem = proj_smem_bytes(a.app.r, e, proj_chunk_rows(a.app.r, e, dspan));
+  static size_t configured = 48 * 1024;
+  if (smem > configured) {
+    cudaError_t err = cudaFuncSetAttribute(lrkv_project_append_kernel<LAT, IO>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    configured = smem;
+  }
+  return launch_pdl(lrkv_project_append_kernel<LAT, IO>, dim3(2 * a.app.Hkv, a.nsplit),
+                    dim3(kProjThreads), smem, st, a);
+}
+
+template <int LAT>
+cudaError_t launch_project_lat(const ProjArgs& a, cudaStream_t st) {
+  return a.app.io_dtype == LRKV_F32 ? launch_project_typed<LAT, LRKV_F32>(a, st)
+                                    : launch_project_typed<LAT, LRKV_BF16>(a, st);
+}
+
 cudaError_t launch_project_append(const ProjArgs& a, cudaStream_t st) {
-  const dim3 grid(2 * a.app.Hkv, a.nsplit), block(kProjThreads);
   switch (a.app.latent_dtype) {
-    case LRKV_F32: return launch_pdl(lrkv_project_append_kernel<LRKV_F32>, grid, block, 0, st, a);
-    case LRKV_BF16: return launch_pdl(lrkv_project_append_kernel<LRKV_BF16>, grid, block, 0, st, a);
-    case LRKV_I8: return launch_pdl(lrkv_project_append_kernel<LRKV_I8>, grid, block, 0, st, a);
-    default: return launch_pdl(lrkv_project_append_kernel<LRKV_E4M3>, grid, block, 0, st, a);
+    case LRKV_F32: return launch_project_lat<LRKV_F32>(a, st);
+    case LRKV_BF16: return launch_project_lat<LRKV_BF16>(a, st);
+    case LRKV_I8: return launch_project_lat<LRKV_I8>(a, st);
+    default: return launch_project_lat<LRKV_E4M3>(a, st);
   }
 }
 
-int project_nsplit(int Hkv, int B, int r, int d_model, size_t workspace_bytes) {
+int project_nsplit(int Hkv, int B, int r, int d_model, int io_bytes, size_t workspace_bytes) {
   if (Hkv > kProjMaxHeads) return 1;
-  int ns = (2 * num_sms() + 2 * Hkv - 1) / (2 * Hkv);
-  ns = std::min(ns, std::max(1, d_model / kProjChunk));
+  // one wave of two CTAs per SM, or more CTAs if a slice would not fit in shared
+  // memory, each with at least kProjMinSpan rows of the factor
+  const int cap = proj_chunk_rows(r, io_bytes, d_model);
+  int ns = std::max(std::max(1, 2 * num_sms() / (2 * Hkv)), (d_model + cap - 1) / cap);
+  ns = std::min(ns, std::max(1, d_model / kProjMinSpan));
   const size_t per = (size_t)2 * Hkv * B * r * sizeof(float);
   const size_t room = workspace_bytes > kHeaderBytes ? workspace_bytes - kHeaderBytes : 0;
   ns = (int)std::min<size_t>((size_t)ns, room / per);

@@ -285,6 +285,23 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
     // counter) is read here or after units handed out from here
     griddep_wait();
     const int BH = a.B * a.Hkv;
+    // split size: the plan's, or the full-length choice scaled by the share of
+    // tiles the rows actually hold (every CTA computes the same), never finer
+    // than the plan's chunk, which bounds the number of splits
+    int chunk = a.chunk, total_units = p.total_units;
+    if (a.device_chunk) {
+      long long tiles = 0;
+      for (int b = lane; b < a.B; b += 32) tiles += (checked_len_tc(a, b) + kT - 1) / kT;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) tiles += __shfl_xor_sync(0xffffffffu, tiles, o);
+      const int tiles_max = max(1, (a.max_seqlen + kT - 1) / kT);
+      const long long full = (long long)a.B * tiles_max;
+      int ct = (int)((a.chunk_hint * tiles + full - 1) / full);
+      ct = max(a.chunk / kT, min(ct, a.chunk_hint));
+      chunk = ct * kT;
+      total_units = ((tiles_max + ct - 1) / ct) * BH;
+      if (blockIdx.x == 0 && lane == 0) atomicExch(a.header + kChunkWord, (unsigned)chunk);
+    }
     uint32_t tile_seq = 0;
     int unit_seq = 0;
     int last_bq_unit = -1;
@@ -293,7 +310,7 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
       int u = 0;
       if (leader) u = (int)atomicAdd(a.header + kWorkCounter, 1u);
       u = __shfl_sync(0xffffffffu, u, 0);
-      const bool term = u >= p.total_units;
+      const bool term = u >= total_units;
       int b = 0, g = 0, s = 0, t0 = 0, t1 = 0;
       if (!term) {
         s = u / BH;
@@ -301,8 +318,8 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
         b = rem / a.Hkv;
         g = rem - b * a.Hkv;
         const int L = checked_len_tc(a, b);
-        t0 = s * a.chunk;
-        t1 = min(L, t0 + a.chunk);
+        t0 = s * chunk;
+        t1 = min(L, t0 + chunk);
         if (t0 >= t1) continue;  // empty split: nothing to do, the merge skips it
       }
       const int us = unit_seq % kUR;

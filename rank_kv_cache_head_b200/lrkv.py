@@ -49,7 +49,8 @@ class Dims(ctypes.Structure):
 class PlanInfo(ctypes.Structure):
     _fields_ = [("algo", ctypes.c_int32), ("num_splits", ctypes.c_int32),
                 ("chunk", ctypes.c_int32), ("grid", ctypes.c_int32),
-                ("smem_bytes", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+                ("smem_bytes", ctypes.c_int32), ("full_chunk", ctypes.c_int32),
+                ("device_chunk", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 _lib = None
@@ -107,7 +108,8 @@ def plan(dims: Dims) -> dict:
         raise LrkvError("lrkv_plan", rc)
     return {"algo": {ALGO_SIMT: "simt", ALGO_TCGEN05: "tcgen05"}[info.algo],
             "num_splits": info.num_splits, "chunk": info.chunk, "grid": info.grid,
-            "smem_bytes": info.smem_bytes}
+            "smem_bytes": info.smem_bytes, "full_chunk": info.full_chunk,
+            "device_chunk": bool(info.device_chunk)}
 
 
 def workspace_bytes(dims: Dims) -> int:

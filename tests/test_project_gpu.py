@@ -25,11 +25,14 @@ def _decode(bits, lat):
 
 
 @pytest.mark.parametrize("ws_bytes", [256, 4 << 20])   # header only: no split; room: split
-@pytest.mark.parametrize("io,lat,r,D", [("f32", "f32", 32, 300), ("bf16", "bf16", 32, 300),
-                                        ("bf16", "bf16", 48, 1000), ("bf16", "i8", 32, 520),
-                                        ("bf16", "e4m3", 64, 2304)])
-def test_project_append_matches_oracle(io, lat, r, D, ws_bytes):
-    B, H, Lcap = 3, 2, 64
+@pytest.mark.parametrize("io,lat,r,D,B", [("f32", "f32", 32, 300, 3), ("bf16", "bf16", 32, 300, 3),
+                                          ("bf16", "bf16", 48, 1000, 3), ("bf16", "i8", 32, 520, 3),
+                                          ("bf16", "e4m3", 64, 2304, 3),
+                                          # several passes of 8 batch rows, ragged last pass
+                                          ("bf16", "bf16", 256, 700, 19), ("f32", "bf16", 8, 1500, 11),
+                                          ("f32", "i8", 144, 2100, 9)])
+def test_project_append_matches_oracle(io, lat, r, D, B, ws_bytes):
+    H, Lcap = 2, 64
     rng = np.random.default_rng(1000 + r + D)
     x = torch.from_numpy(rng.standard_normal((B, D))).to(_IO[io])
     AK = torch.from_numpy(rng.standard_normal((H, D, r)) / math.sqrt(D)).to(_IO[io])
@@ -43,7 +46,7 @@ def test_project_append_matches_oracle(io, lat, r, D, ws_bytes):
         Z0 = Z0.to(_LAT[lat])
     quant = lat in ("i8", "e4m3")
     S0 = torch.from_numpy(rng.uniform(0.5, 1.5, (2, B, H, Lcap)).astype(np.float32)) if quant else None
-    seq0 = torch.tensor([5, Lcap - 1, Lcap], dtype=torch.int32)
+    seq0 = torch.tensor([5, Lcap - 1, Lcap] + [(7 * b) % (Lcap + 1) for b in range(3, B)], dtype=torch.int32)
 
     dims = lrkv.make_dims(B, H, H, 128, r, Lcap, Lcap, io, lat)
     ZK, ZV = Z0[0].clone().cuda(), Z0[1].clone().cuda()
