@@ -44,7 +44,7 @@ from rank_kv_cache_head_b200 import lrkv  # noqa: E402
 from rank_kv_cache_head_b200.metrics import (ClockSampler, max_over_ranks,  # noqa: E402
                                              step_bytes, sum_over_ranks)
 from rank_kv_cache_head_b200.workloads import (WORKLOADS, make_append_rows,  # noqa: E402
-                                               make_inputs, seqlens_for)
+                                               make_inputs, seqlens_for, with_text_factors)
 
 METRIC = "low-rank decode attention: latent GB/s, tokens/s/GPU, % of HBM roofline"
 UNIT = "GB/s"
@@ -67,6 +67,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--projection-dmodel", type=int, default=4096,
                     help="also time lrkv_project_append with this hidden size (0: skip)")
+    ap.add_argument("--n-visual", type=int, default=0, metavar="P",
+                    help="modality-separated factors: positions < P use a visual factor "
+                         "set, the rest a text set (0: one set, the default)")
     ap.add_argument("--profile", type=int, default=0, metavar="N",
                     help="no timing: run N eager decode-attention calls on one cache copy "
                          "and exit (a short, fixed launch sequence for ncu captures)")
@@ -150,7 +153,7 @@ def blas_threads() -> int:
 # ---------------------------------------------------------------------------------------
 
 
-def oracle_sample(wl, inputs, budget_s: float, max_units=None, rng_seed=0):
+def oracle_sample(wl, inputs, budget_s: float, max_units=None, rng_seed=0, n_visual=0):
     """Time the fp64 oracle on whole (batch row, KV head) units in a seeded random
     order until ``budget_s`` seconds of work are done. Returns (seconds per unit,
     units timed, latent bytes timed, seconds)."""
@@ -178,8 +181,12 @@ def oracle_sample(wl, inputs, budget_s: float, max_units=None, rng_seed=0):
         if inputs["ZK_scale"] is not None:
             SK = inputs["ZK_scale"][b:b + 1, g:g + 1, :Lb].numpy().astype(np.float64)
             SV = inputs["ZV_scale"][b:b + 1, g:g + 1, :Lb].numpy().astype(np.float64)
-        orc.decode_attention(q[b:b + 1, g * G:(g + 1) * G], ZK, ZV, BK[g:g + 1], BV[g:g + 1],
-                             np.array([Lb]), SK, SV)
+        if n_visual:     # factors [2][Hkv][r][d]: both sets of this head
+            orc.decode_attention(q[b:b + 1, g * G:(g + 1) * G], ZK, ZV, BK[:, g:g + 1],
+                                 BV[:, g:g + 1], np.array([Lb]), SK, SV, n_visual=n_visual)
+        else:
+            orc.decode_attention(q[b:b + 1, g * G:(g + 1) * G], ZK, ZV, BK[g:g + 1], BV[g:g + 1],
+                                 np.array([Lb]), SK, SV)
         spent += time.perf_counter() - t0
         n += 1
         lat_bytes += Lb * per_tok
@@ -323,13 +330,15 @@ def run_ours(args, rank, world, local):
     Lmax = int(target.max())
     capacity = ((Lmax + args.e2e_steps + 16 + 7) // 8) * 8
     inputs = make_inputs(wl, capacity=capacity, seqlens=target)
-    sb = step_bytes(wl, target)
+    if args.n_visual:
+        inputs = with_text_factors(wl, inputs)
+    sb = step_bytes(wl, target, factor_sets=2 if args.n_visual else 1)
     per_copy = sb["latent"] + sb["scales"]
     n_copies = max(2, math.ceil(3 * L2_BYTES / max(per_copy, 1)))
     n_copies = min(n_copies, 64)
 
     dims = lrkv.make_dims(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.d_head, wl.rank, capacity,
-                          Lmax, wl.io_dtype, wl.latent_dtype, 0, args.algo)
+                          Lmax, wl.io_dtype, wl.latent_dtype, 0, args.algo, n_visual=args.n_visual)
     plan = lrkv.plan(dims)
     q = inputs["q"].to(dev)
     BK, BV = inputs["BK"].to(dev), inputs["BV"].to(dev)
@@ -440,7 +449,7 @@ def run_ours(args, rank, world, local):
     # the end-to-end steps keep appending, so their planning hint covers the growth
     dims_e2e = lrkv.make_dims(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.d_head, wl.rank,
                               capacity, min(capacity, Lmax + ke // n_copies + 1), wl.io_dtype,
-                              wl.latent_dtype, 0, args.algo)
+                              wl.latent_dtype, 0, args.algo, n_visual=args.n_visual)
     ws_e2e = lrkv.new_workspace(dims_e2e, device=dev)
     uses = [0] * n_copies
     e2e_lat = 0
@@ -492,6 +501,9 @@ def run_ours(args, rank, world, local):
             "" if wl.latent_dtype in ("bf16", "f32") else f"+{wl.latent_dtype}-latents"),
         "data": "synthetic (seeded; shapes and distributions of the workload definition)",
         "config": dict(workload_config(wl, target, plan, plan["algo"]),
+                       **({"n_visual": args.n_visual,
+                           "factors": "modality-separated (visual set below n_visual, text set after)"}
+                          if args.n_visual else {}),
                        parallelism=f"dp{world} (independent batches per GPU)",
                        l2=f"cache rotated over {n_copies} copies ({n_copies * per_copy / 1e6:.0f} MB "
                           f">= 3x L2) between uses"),
@@ -513,7 +525,7 @@ def run_ours(args, rank, world, local):
     if args.projection_dmodel > 0:
         line["project_append"] = measure_projection(wl, dev, args.projection_dmodel)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        per_unit, n, lb, spent = oracle_sample(wl, inputs, args.cpu_seconds)
+        per_unit, n, lb, spent = oracle_sample(wl, inputs, args.cpu_seconds, n_visual=args.n_visual)
         cores = blas_threads()
         cpu_val = lb / spent / 1e9
         line["cpu_baseline"] = {

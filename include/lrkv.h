@@ -37,6 +37,7 @@
  *   ZK, ZV          [B][Hkv][Lc][r]     latent_dtype (int8 codes, or e4m3 bytes)
  *   ZK_scale/ZV_scale [B][Hkv][Lc]      fp32, one per token (I8/E4M3 only)
  *   BK, BV          [Hkv][r][d]         io_dtype
+ *                   [2][Hkv][r][d] when n_visual > 0 (visual set, then text set)
  *   seqlens         [B]                 int32, valid positions per row
  *   lse_out         [B][Hq]             fp32, natural log (optional)
  */
@@ -50,7 +51,7 @@
 extern "C" {
 #endif
 
-#define LRKV_VERSION 1
+#define LRKV_VERSION 2
 
 /* element types */
 typedef enum {
@@ -95,7 +96,14 @@ typedef enum {
  *  latent_dtype: any lrkv_dtype (F32 latents require F32 io);
  *  num_splits: 0 = choose automatically, else the split count to use (clamped to
  *      the number of 128-token tiles of max_seqlen);
- *  algo: an lrkv_algo.
+ *  algo: an lrkv_algo;
+ *  n_visual: 0 = one factor set. Otherwise modality-separated factors
+ *      ("AttentionPack", Metodologia 2.A: visual and text tokens are compressed
+ *      separately, their distributions differ): positions [0, n_visual) of every
+ *      row are rebuilt with the first (visual) factor set and positions >= n_visual
+ *      with the second (text) set, BK/BV [2][Hkv][r][d]. A multiple of 16 in
+ *      [0, max_seq]. The split size is chosen as without it; splits are then laid
+ *      out over the two segments separately, so none straddles the boundary.
  */
 typedef struct {
   int32_t batch;
@@ -109,6 +117,7 @@ typedef struct {
   int32_t latent_dtype;
   int32_t num_splits;
   int32_t algo;
+  int32_t n_visual;
 } lrkv_dims;
 
 /* What lrkv_decode_attn will do for these dims (for tests and benchmarks). */
@@ -212,11 +221,10 @@ int lrkv_decode_step_host(const lrkv_dims* dims, const void* q_host, const void*
  * int8 / e4m3 codes with a per-row fp32 absmax scale), then seqlens[b] += 1.
  *   x      [B][d_model], io dtype, device
  *   AK, AV [H_kv][d_model][rank], io dtype, device, 16-byte aligned
- *   other arguments as lrkv_append. The workspace needs its 256-byte header; the
- *   bytes after it, when there are enough (a decode workspace of the same dims
- *   usually has), hold partial sums so the hidden size is split over more CTAs.
- *   The sums are added in a fixed order, so a call is deterministic for a given
- *   workspace size (different sizes may split differently and round differently).
+ *   other arguments as lrkv_append. Only the workspace's 256-byte header is used.
+ *   The hidden size is split over up to 8 CTAs per factor (one thread-block
+ *   cluster) that add their partial sums through distributed shared memory in a
+ *   fixed order, so a call is deterministic.
  * Errors: LRKV_ERR_DIMS (dims, d_model outside [1, 2^20]), LRKV_ERR_ARG (NULL pointer,
  * scales present iff quantised latents), LRKV_ERR_ALIGN, LRKV_ERR_WORKSPACE,
  * LRKV_ERR_LAUNCH. A row whose slot is past the capacity is left untouched, keeps its

@@ -145,13 +145,19 @@ def dequantise(Z: np.ndarray, scale) -> np.ndarray:
 
 
 def decode_attention(q, ZK, ZV, BK, BV, seqlens, ZK_scale=None, ZV_scale=None,
-                     score_shift: float = 0.0, pairs=None):
+                     score_shift: float = 0.0, pairs=None, n_visual: int = 0):
     """Single-token decode attention over a per-head low-rank cache, in float64.
 
     q [B][Hq][d]; ZK, ZV [B][Hkv][L_cap][r] (decoded codes); scales [B][Hkv][L_cap]
     or None; BK, BV [Hkv][r][d]; seqlens [B]. Returns out [B][Hq][d], lse [B][Hq]
     (natural log). ``score_shift`` adds a constant to every score (used only to pin
     the softmax stabilisation). ``pairs`` restricts the work to some (b, h).
+
+    Modality-separated factors ("AttentionPack", Metodologia 2.A: visual and text
+    tokens are compressed separately because their distributions differ): with
+    n_visual > 0, BK and BV are [2][Hkv][r][d]; positions t < n_visual of every row
+    are rebuilt with the first (visual) set and positions t >= n_visual with the
+    second (text) set. Reading: one boundary shared by every row, visual tokens first.
     """
     q = np.asarray(q, np.float64)
     B, Hq, d = q.shape
@@ -170,8 +176,15 @@ def decode_attention(q, ZK, ZV, BK, BV, seqlens, ZK_scale=None, ZV_scale=None,
             sv = None if ZV_scale is None else ZV_scale[b, g, :Lb]
             Zk = dequantise(np.asarray(ZK[b, g, :Lb, :], np.float64), sk)
             Zv = dequantise(np.asarray(ZV[b, g, :Lb, :], np.float64), sv)
-            K = Zk @ np.asarray(BK[g], np.float64)       # Lb x d, rebuilt keys
-            V = Zv @ np.asarray(BV[g], np.float64)       # Lb x d, rebuilt values
+            if n_visual > 0:
+                P = min(n_visual, Lb)                    # visual rows, then text rows
+                K = np.concatenate([Zk[:P] @ np.asarray(BK[0][g], np.float64),
+                                    Zk[P:] @ np.asarray(BK[1][g], np.float64)])
+                V = np.concatenate([Zv[:P] @ np.asarray(BV[0][g], np.float64),
+                                    Zv[P:] @ np.asarray(BV[1][g], np.float64)])
+            else:
+                K = Zk @ np.asarray(BK[g], np.float64)   # Lb x d, rebuilt keys
+                V = Zv @ np.asarray(BV[g], np.float64)   # Lb x d, rebuilt values
             for h in heads:
                 s = (K @ q[b, h]) / math.sqrt(d) + score_shift
                 m = s.max()

@@ -46,6 +46,7 @@ int check_dims(const lrkv_dims* d) {
   if (d->rank < 8 || d->rank > 256 || d->rank % 8 != 0) return LRKV_ERR_DIMS;
   if (d->max_seq < 1 || d->max_seqlen < 0 || d->max_seqlen > d->max_seq) return LRKV_ERR_DIMS;
   if (d->num_splits < 0) return LRKV_ERR_DIMS;
+  if (d->n_visual < 0 || d->n_visual > d->max_seq || d->n_visual % 16 != 0) return LRKV_ERR_DIMS;
   if (d->io_dtype != LRKV_F32 && d->io_dtype != LRKV_BF16) return LRKV_ERR_DTYPE;
   if (d->latent_dtype < LRKV_F32 || d->latent_dtype > LRKV_E4M3) return LRKV_ERR_DTYPE;
   if (d->latent_dtype == LRKV_F32 && d->io_dtype != LRKV_F32) return LRKV_ERR_DTYPE;
@@ -140,8 +141,8 @@ int make_plan(const lrkv_dims* d, Plan* p) {
     p->device_chunk = 1;
     chunk_tiles = (chunk_tiles + 3) / 4;
   }
-  p->S = (tiles_max + chunk_tiles - 1) / chunk_tiles;
   p->chunk = chunk_tiles * kTile;
+  p->S = total_splits(d->n_visual, d->max_seqlen, p->chunk);
   if (p->algo == LRKV_ALGO_TCGEN05) {
     p->smem = tc_smem;
     p->grid = std::min(P, rows * p->S);
@@ -271,6 +272,7 @@ int lrkv_decode_attn_timed(const lrkv_dims* dims, const void* q, const void* ZK,
   a.max_seqlen = dims->max_seqlen;
   a.S = p.S;
   a.chunk = p.chunk;
+  a.n_visual = dims->n_visual;
   a.io_dtype = dims->io_dtype;
   a.latent_dtype = dims->latent_dtype;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_head));
@@ -307,6 +309,7 @@ int lrkv_decode_attn_timed(const lrkv_dims* dims, const void* q, const void* ZK,
   m.d = a.d;
   m.S = p.S;
   m.chunk = p.chunk;
+  m.n_visual = a.n_visual;
   m.Lcap = a.Lcap;
   m.max_seqlen = a.max_seqlen;
   m.io_dtype = a.io_dtype;

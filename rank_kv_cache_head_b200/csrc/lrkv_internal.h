@@ -21,6 +21,35 @@ enum HeaderWord {
   kProjHeadWord = 8,   // words 8..63: per-KV-head counters of the projection
 };
 
+// Split layout. A row is two segments when the factors are modality-separated:
+// [0, n_visual) rebuilt with the visual set and [n_visual, L) with the text set
+// (one segment [0, L) otherwise, n_visual = 0). Each segment is cut into splits of
+// `chunk` tokens; the visual splits come first. No split straddles the boundary.
+__host__ __device__ inline int visual_splits(int n_visual, int max_seqlen, int chunk) {
+  const int P = n_visual < max_seqlen ? n_visual : max_seqlen;
+  return (P + chunk - 1) / chunk;
+}
+__host__ __device__ inline int total_splits(int n_visual, int max_seqlen, int chunk) {
+  const int rest = max_seqlen > n_visual ? max_seqlen - n_visual : 0;
+  const int S = visual_splits(n_visual, max_seqlen, chunk) + (rest + chunk - 1) / chunk;
+  return S > 0 ? S : 1;
+}
+// Token range [t0, t1) of split s in a row of length L (empty when t0 >= t1), and
+// the factor set it uses (0 visual / single set, 1 text).
+__host__ __device__ inline int split_range(int s, int L, int n_visual, int max_seqlen, int chunk,
+                                           int* t0, int* t1) {
+  const int sv = visual_splits(n_visual, max_seqlen, chunk);
+  if (s < sv) {
+    *t0 = s * chunk;
+    const int end = L < n_visual ? L : n_visual;
+    *t1 = end < *t0 + chunk ? end : *t0 + chunk;
+    return 0;
+  }
+  *t0 = n_visual + (s - sv) * chunk;
+  *t1 = L < *t0 + chunk ? L : *t0 + chunk;
+  return n_visual > 0 ? 1 : 0;
+}
+
 // Launch plan for one call (depends only on dims and the device).
 struct Plan {
   int algo;         // LRKV_ALGO_SIMT or LRKV_ALGO_TCGEN05
@@ -54,6 +83,7 @@ struct SplitArgs {
   int debug_stall;   // test hook: work unit 0's first tile is withheld (see lrkv.h)
   int device_chunk;  // choose the split size on the device (chunk = the finest, S its bound)
   int chunk_hint;    // device_chunk: the split size, in tiles, for rows at full length
+  int n_visual;      // > 0: modality-separated factors, BK/BV [2][Hkv][r][d]
 };
 
 struct MergeArgs {
@@ -65,6 +95,7 @@ struct MergeArgs {
   uint32_t* header;
   int B, Hq, d, S, chunk, Lcap, max_seqlen;
   int io_dtype;
+  int n_visual;      // split layout (see split_range)
   int device_chunk;  // read the split size the split kernel chose from the header
 };
 

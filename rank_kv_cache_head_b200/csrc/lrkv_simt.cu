@@ -72,8 +72,8 @@ __global__ void __launch_bounds__(kSimtThreads) lrkv_split_simt(SplitArgs a) {
   const int d = a.d, r = a.r, G = a.G, T = kSimtTile;
 
   const int L = checked_len(a.seqlens, b, a.Lcap, a.max_seqlen, a.header, false);
-  const int t_begin = s * a.chunk;
-  const int t_end = min(L, t_begin + a.chunk);
+  int t_begin, t_end;
+  const int fset = split_range(s, L, a.n_visual, a.max_seqlen, a.chunk, &t_begin, &t_end);
   if (t_begin >= t_end) return;  // empty split: the merge skips it
 
   float* bk = sm;                 // [r][d]
@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(kSimtThreads) lrkv_split_simt(SplitArgs a) {
   float* ls = ms + G;             // [G] running sum
   float* al = ls + G;             // [G] rescale factor of the current tile
 
-  const size_t fac_base = (size_t)g * r * d;
+  const size_t fac_base = ((size_t)fset * a.Hkv + g) * r * d;   // factor set, then head
   for (int i = tid; i < r * d; i += kSimtThreads) {
     bk[i] = load_io(a.BK, fac_base + i, a.io_dtype);
     bv[i] = load_io(a.BV, fac_base + i, a.io_dtype);
@@ -217,19 +217,36 @@ __global__ void __launch_bounds__(128) lrkv_merge(MergeArgs a) {
   // the split size: the plan's, or the one the tensor-core split kernel chose
   const int chunk = a.device_chunk ? (int)*reinterpret_cast<volatile uint32_t*>(a.header + kChunkWord)
                                    : a.chunk;
-  const int ns = min(a.S, (L + chunk - 1) / chunk);
+  // the row's non-empty splits, in order: the first n1 are physical splits 0..n1-1
+  // (the visual segment, or the whole row), the rest start at physical split sv
+  // (the text segment of modality-separated factors)
+  int ns, n1, sv = 0;
+  if (a.n_visual > 0) {
+    sv = visual_splits(a.n_visual, a.max_seqlen, chunk);
+    n1 = (min(L, a.n_visual) + chunk - 1) / chunk;
+    ns = min(a.S, n1 + (max(0, L - a.n_visual) + chunk - 1) / chunk);
+  } else {
+    ns = min(a.S, (L + chunk - 1) / chunk);
+    n1 = ns;
+  }
+  auto phys = [&](int j) { return j < n1 ? j : sv + (j - n1); };
+  // the prefetched values are physical splits 0..: reload the ones past n1
+  if (tid < 32 && lane >= n1 && lane < ns) lse0 = lse[phys(lane)];
+#pragma unroll
+  for (int k = 0; k < kPre; ++k)
+    if (active && k >= n1 && k < ns) opre[k] = o[(size_t)phys(k) * a.d + tid];
   if (tid < 32) {
     float mx = lane < ns ? lse0 : -CUDART_INF_F;
-    for (int s = lane + 32; s < ns; s += 32) mx = fmaxf(mx, lse[s]);
+    for (int s = lane + 32; s < ns; s += 32) mx = fmaxf(mx, lse[phys(s)]);
 #pragma unroll
     for (int k = 16; k > 0; k >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, k));
     float tot = lane < ns ? expf(lse0 - mx) : 0.f;
-    for (int s = lane + 32; s < ns; s += 32) tot += expf(lse[s] - mx);
+    for (int s = lane + 32; s < ns; s += 32) tot += expf(lse[phys(s)] - mx);
 #pragma unroll
     for (int k = 16; k > 0; k >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, k);
     const float LSE = (ns > 0) ? mx + logf(tot) : -CUDART_INF_F;
     if (lane < ns) wsm[lane] = expf(lse0 - LSE);
-    for (int s = lane + 32; s < ns; s += 32) wsm[s] = expf(lse[s] - LSE);
+    for (int s = lane + 32; s < ns; s += 32) wsm[s] = expf(lse[phys(s)] - LSE);
     if (a.lse_out && lane == 0) a.lse_out[bh] = LSE;
   }
   __syncthreads();
@@ -241,9 +258,9 @@ __global__ void __launch_bounds__(128) lrkv_merge(MergeArgs a) {
   int s = kPre;
   for (; s + 4 <= ns; s += 4) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) v[k] = fmaf(wsm[s + k], o[(size_t)(s + k) * a.d + tid], v[k]);
+    for (int k = 0; k < 4; ++k) v[k] = fmaf(wsm[s + k], o[(size_t)phys(s + k) * a.d + tid], v[k]);
   }
-  for (; s < ns; ++s) v[0] = fmaf(wsm[s], o[(size_t)s * a.d + tid], v[0]);
+  for (; s < ns; ++s) v[0] = fmaf(wsm[s], o[(size_t)phys(s) * a.d + tid], v[0]);
   const float r = (v[0] + v[1]) + (v[2] + v[3]);
   const size_t oi = (size_t)bh * a.d + tid;
   if (a.io_dtype == LRKV_F32) static_cast<float*>(a.out)[oi] = r;
@@ -346,35 +363,73 @@ __global__ void __launch_bounds__(1024) lrkv_append_kernel(AppendArgs a) {
 // e4m3 codes with a per-row absmax scale). The last CTA to finish advances seqlens.
 // grid (2 Hkv, nsplit): CTA = (KV head, K | V, slice of the hidden size), 256
 // threads. One thread issues a bulk copy of the CTA's factor rows into shared memory
-// (they are contiguous in A) while the others stage rows of x as fp32, so the factor
-// crosses HBM once and every later pass over the batch reads it from shared memory.
-// A factor row (r columns) is read by tpr lanes, 8 columns each (tpr = r / 8 rounded up
-// to a power of two); the other lanes of the warp and the 8 warps take other rows.
-// Each thread keeps 8 batch rows x 8 columns of fp32 sums in packed pairs
-// (fma.rn.f32x2). The sums are reduced over the lanes that share columns (a butterfly
-// in which each step halves the values a lane holds), then over the warps in a fixed
-// order. With nsplit > 1 every CTA writes its partial sums to the workspace and the
-// last CTA of a KV head adds them in a fixed order and writes that head's rows
-// (deterministic). A slice larger than the shared-memory budget is taken in chunks,
-// copied again for every pass.
+// (they are contiguous in A) while the others stage a block of rows of x as fp32
+// (16-byte loads where x allows), so the factor crosses HBM once and every pass over
+// the batch reads both operands from shared memory. A factor row (r columns) is read
+// by tpr lanes, 8 columns each (tpr = r / 8 rounded up to a power of two); the other
+// lanes of the warp and the 8 warps take other rows. Each thread keeps 8 batch rows x
+// 8 columns of fp32 sums in packed pairs (fma.rn.f32x2). The sums are reduced over the
+// lanes that share columns (a butterfly in which each step halves the values a lane
+// holds), then over the warps in a fixed order. With nsplit > 1 every CTA writes its
+// partial sums to the workspace and the last CTA of a KV head adds them in a fixed
+// order and writes that head's rows (deterministic). A slice larger than the
+// shared-memory budget is taken in chunks, copied again for every pass of 8 rows.
 constexpr int kProjThreads = 256;
 constexpr int kProjWarps = kProjThreads / 32;
 constexpr int kProjRows = 8;              // batch rows per pass
 constexpr int kProjMaxChunk = 1024;       // factor rows staged at a time, at most
 constexpr int kProjABytes = 64 * 1024;    // shared-memory budget for factor rows
+constexpr int kProjSmemTarget = 110 * 1024;  // two CTAs per SM
 constexpr int kProjMinSpan = 64;          // fewest hidden-size rows a CTA takes when splitting
-constexpr int kProjMaxHeads = 56;         // per-head counters live in header words 8..63
+constexpr int kProjMaxCluster = 8;        // CTAs sharing one factor: one portable cluster
+constexpr int kProjClusterBytes = 32 * 1024;  // a CTA's partial sums [B][r] must fit this
 
-// factor rows a CTA stages at a time, for row width r and element size e
+// hidden-size rows per CTA: a multiple of 8, so 16-byte loads of x stay aligned
+__host__ __device__ inline int proj_dspan(int D, int ns) { return ((D + ns - 1) / ns + 7) / 8 * 8; }
+
+// factor rows a CTA stages at a time (a multiple of 8), for row width r, element size e
 __host__ __device__ inline int proj_chunk_rows(int r, int e, int dspan) {
-  const int cap = min(kProjMaxChunk, kProjABytes / (r * e));
-  return max(1, min(cap, dspan));
+  const int cap = min(kProjMaxChunk, kProjABytes / (r * e)) / 8 * 8;
+  return max(8, min(cap, dspan));
 }
 
-// dynamic shared memory: barrier, factor rows, x rows (or the warps' partial sums), sums
-__host__ __device__ inline size_t proj_smem_bytes(int r, int e, int cr) {
-  const size_t xs = (size_t)kProjRows * cr, red = (size_t)kProjWarps * kProjRows * r;
-  return 16 + (size_t)cr * r * e + sizeof(float) * ((xs > red ? xs : red) + (size_t)kProjRows * r);
+// batch rows of x staged at once (a multiple of 8): as many as the budget holds when
+// the slice is resident, 8 when it is taken in chunks
+__host__ __device__ inline int proj_batch_block(int B, int r, int e, int cr, bool chunked, int ns) {
+  const int b8 = (B + 7) / 8 * 8;
+  if (chunked) return 8;
+  const long long room = (long long)kProjSmemTarget - 16 - (long long)cr * r * e -
+                         (long long)(kProjWarps + 1) * kProjRows * r * 4 -
+                         (ns > 1 ? (long long)B * r * 4 : 0);
+  const int rows = (int)(room > 0 ? room / (cr * 4) : 0) / 8 * 8;
+  return max(8, min(rows, b8));
+}
+
+// dynamic shared memory: barrier, factor rows, x rows, the warps' partial sums, sums,
+// and with a split hidden size this CTA's partial sums of every batch row
+__host__ __device__ inline size_t proj_smem_bytes(int B, int r, int e, int cr, int bblk, int ns) {
+  return 16 + (size_t)cr * r * e +
+         sizeof(float) * ((size_t)bblk * cr + (size_t)(kProjWarps + 1) * kProjRows * r +
+                          (ns > 1 ? (size_t)B * r : 0));
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// fp32 at a shared-memory address of another CTA of the cluster
+__device__ __forceinline__ float ld_cluster_f32(uint32_t local_addr, uint32_t rank) {
+  uint32_t remote;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
 }
 
 template <int LAT>
@@ -414,6 +469,66 @@ __device__ __forceinline__ void proj_row8(const char* p, uint64_t (&a2)[4]) {
   }
 }
 
+// xs[row][i] = x[b0 + row][d0 + i] as fp32 for row < srows, i < cr; zero past nrows
+// rows or dn columns. vec: x rows and d0 are 16-byte aligned and dn, cr are multiples
+// of 8, so every thread moves 16-byte words, eight in flight.
+template <int IO>
+__device__ __forceinline__ void proj_stage_x(float* xs, const void* x, int b0, int nrows,
+                                             int srows, int D, int d0, int dn, int cr, int t,
+                                             bool vec) {
+  constexpr int E = IO == LRKV_F32 ? 4 : 2;
+  constexpr int V = 16 / E;                          // elements a 16-byte word
+  const char* xb = static_cast<const char*>(x);
+  if (vec) {
+    const int wpr = cr / V, total = srows * wpr;
+    for (int w0 = t; w0 < total; w0 += 8 * kProjThreads) {
+      uint4 buf[8];
+      int row = w0 / wpr, iw = w0 - row * wpr;       // advanced by kProjThreads words
+      const int drow = kProjThreads / wpr, diw = kProjThreads - drow * wpr;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int w = w0 + k * kProjThreads, i = iw * V;
+        buf[k] = make_uint4(0u, 0u, 0u, 0u);
+        if (w < total && row < nrows && i < dn)
+          buf[k] = __ldg(reinterpret_cast<const uint4*>(xb + ((size_t)(b0 + row) * D + d0 + i) * E));
+        row += drow;
+        iw += diw;
+        if (iw >= wpr) { iw -= wpr; ++row; }
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int w = w0 + k * kProjThreads;
+        if (w >= total) continue;
+        // xs is [row][cr] and a row holds wpr words: word w starts at element w * V
+        float4* o = reinterpret_cast<float4*>(xs + (size_t)w * V);
+        if constexpr (IO == LRKV_F32) {
+          o[0] = make_float4(__uint_as_float(buf[k].x), __uint_as_float(buf[k].y),
+                             __uint_as_float(buf[k].z), __uint_as_float(buf[k].w));
+        } else {
+          o[0] = make_float4(__uint_as_float(buf[k].x << 16), __uint_as_float(buf[k].x & 0xffff0000u),
+                             __uint_as_float(buf[k].y << 16), __uint_as_float(buf[k].y & 0xffff0000u));
+          o[1] = make_float4(__uint_as_float(buf[k].z << 16), __uint_as_float(buf[k].z & 0xffff0000u),
+                             __uint_as_float(buf[k].w << 16), __uint_as_float(buf[k].w & 0xffff0000u));
+        }
+      }
+    }
+  } else {
+    const int total = srows * cr;
+    for (int e0 = t; e0 < total; e0 += 8 * kProjThreads) {
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int e = e0 + k * kProjThreads;
+        const int row = e / cr, i = e - row * cr;
+        v[k] = (e < total && row < nrows && i < dn) ? load_io(x, (size_t)(b0 + row) * D + d0 + i, IO) : 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (e0 + k * kProjThreads < total) xs[e0 + k * kProjThreads] = v[k];
+    }
+  }
+}
+
 template <int LAT, int IO>
 __global__ void __launch_bounds__(kProjThreads, 2) lrkv_project_append_kernel(ProjArgs pa) {
   constexpr int E = IO == LRKV_F32 ? 4 : 2;          // bytes an element
@@ -421,21 +536,25 @@ __global__ void __launch_bounds__(kProjThreads, 2) lrkv_project_append_kernel(Pr
   extern __shared__ __align__(16) unsigned char proj_smem[];
   __shared__ int abort_flag;
   const AppendArgs& a = pa.app;
-  const int r = a.r;
+  const int r = a.r, B = a.B;
   const int gk = blockIdx.x, g = gk >> 1, kv = gk & 1, sp = blockIdx.y, ns = pa.nsplit;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int D = pa.d_model;
-  const int dspan = (D + ns - 1) / ns;
+  const int dspan = proj_dspan(D, ns);
   const int dlo = min(D, sp * dspan), dhi = min(D, dlo + dspan);
   const int cr = proj_chunk_rows(r, E, dspan);
   const int nchunks = max(1, (dhi - dlo + cr - 1) / cr);
   const bool resident = nchunks == 1;
+  // the launch's shared memory is sized for the longest slice, so the block of batch
+  // rows depends on that slice, not on this CTA's (the last one may be shorter)
+  const int bblk = proj_batch_block(B, r, E, cr, min(dspan, D) > cr, ns);
+  const bool vec = (D % 8 == 0) && ((reinterpret_cast<uintptr_t>(pa.x) & 15) == 0);
   const uint32_t bar = smem_addr(proj_smem);
   char* As = reinterpret_cast<char*>(proj_smem + 16);              // [row][r] as in A
   float* xs = reinterpret_cast<float*>(As + (size_t)cr * r * E);   // [batch row][row]
-  float* red = xs;                                                 // [warp][batch row][col]
-  const size_t xs_floats = (size_t)kProjRows * cr, red_floats = (size_t)kProjWarps * kProjRows * r;
-  float* zs = xs + (xs_floats > red_floats ? xs_floats : red_floats);   // [batch row][col]
+  float* red = xs + (size_t)bblk * cr;                             // [warp][batch row][col]
+  float* zs = red + kProjWarps * kProjRows * r;                    // [batch row][col]
+  float* zc = zs + kProjRows * r;              // ns > 1: this CTA's partial sums [B][r]
   const char* A = static_cast<const char*>(kv ? pa.AV : pa.AK) + (size_t)g * D * r * E;
   const size_t row_bytes = (size_t)r * E;
   if (t == 0) {
@@ -463,86 +582,91 @@ __global__ void __launch_bounds__(kProjThreads, 2) lrkv_project_append_kernel(Pr
   const int nslots = kProjWarps * spw, slot = warp * spw + lane / tpr;
   const bool active = c0 < r;
 
-  for (int b0 = 0; b0 < a.B; b0 += kProjRows) {
-    const int nb = min(kProjRows, a.B - b0);
-    uint64_t acc[kProjRows][4];
+  for (int blk0 = 0; blk0 < B; blk0 += bblk) {
+    const int nblk = min(bblk, B - blk0);
+    for (int g8 = 0; g8 < nblk; g8 += kProjRows) {
+      const int b0 = blk0 + g8, nb = min(kProjRows, nblk - g8);
+      uint64_t acc[kProjRows][4];
 #pragma unroll
-    for (int bb = 0; bb < kProjRows; ++bb)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[bb][j] = 0ull;
-    for (int ch = 0; ch < nchunks; ++ch) {
-      const int d0 = dlo + ch * cr, dn = min(cr, dhi - d0);
-      __syncthreads();                           // the previous chunk / pass is consumed
-      if (!resident) issue(d0, dn);
       for (int bb = 0; bb < kProjRows; ++bb)
-        for (int i = t; i < cr; i += kProjThreads)
-          xs[bb * cr + i] = (bb < nb && i < dn) ? load_io(pa.x, (size_t)(b0 + bb) * D + d0 + i, IO) : 0.f;
-      __syncthreads();
-      if (dn > 0 && !mbar_wait(bar, (copies - 1) & 1, &abort_flag, kWaitNs)) timed_out = true;
-      if (active) {
-        for (int i = slot; i < dn; i += nslots) {
-          uint64_t a2[4];
-          proj_row8<IO>(As + (size_t)i * row_bytes + (size_t)c0 * E, a2);
 #pragma unroll
-          for (int bb = 0; bb < kProjRows; ++bb) {
-            const float xv = xs[bb * cr + i];
-            const uint64_t x2 = pack2(xv, xv);
+        for (int j = 0; j < 4; ++j) acc[bb][j] = 0ull;
+      for (int ch = 0; ch < nchunks; ++ch) {
+        const int d0 = dlo + ch * cr, dn = min(cr, dhi - d0);
+        if (!resident || g8 == 0) {
+          // resident slice: the block's x rows once; chunked: this pass's rows per chunk
+          __syncthreads();                       // earlier readers of xs / As are done
+          if (!resident) issue(d0, dn);
+          if (resident) proj_stage_x<IO>(xs, pa.x, blk0, nblk, bblk, D, d0, dn, cr, t, vec);
+          else proj_stage_x<IO>(xs, pa.x, b0, nb, kProjRows, D, d0, dn, cr, t, vec);
+          __syncthreads();
+          if (dn > 0 && !mbar_wait(bar, (copies - 1) & 1, &abort_flag, kWaitNs)) timed_out = true;
+        }
+        const float* xg = xs + (size_t)(resident ? g8 : 0) * cr;
+        if (active) {
+          for (int i = slot; i < dn; i += nslots) {
+            uint64_t a2[4];
+            proj_row8<IO>(As + (size_t)i * row_bytes + (size_t)c0 * E, a2);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[bb][j] = ffma2p(x2, a2[j], acc[bb][j]);
+            for (int bb = 0; bb < kProjRows; ++bb) {
+              const float xv = xg[bb * cr + i];
+              const uint64_t x2 = pack2(xv, xv);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) acc[bb][j] = ffma2p(x2, a2[j], acc[bb][j]);
+            }
           }
         }
       }
-    }
-    // lanes that share columns: each butterfly step sends half of the values a lane
-    // holds to its partner and keeps the other half, so after s steps a lane holds
-    // 64 / 2^s sums; which ones depends on the lane's bits (index base `off`)
-    float v[64];
+      // lanes that share columns: each butterfly step sends half of the values a lane
+      // holds to its partner and keeps the other half, so after s steps a lane holds
+      // 64 / 2^s sums; which ones depends on the lane's bits (index base `off`)
+      float v[64];
 #pragma unroll
-    for (int bb = 0; bb < kProjRows; ++bb)
+      for (int bb = 0; bb < kProjRows; ++bb)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = unpack2(acc[bb][j]);
-        v[bb * 8 + 2 * j] = f.x;
-        v[bb * 8 + 2 * j + 1] = f.y;
-      }
-    int off = 0, held = 64;
-#pragma unroll
-    for (int s = 0; s < 5; ++s) {
-      const int h = 32 >> s;                     // values sent (and kept) in this step
-      const int o = tpr << s;
-      if (o < 32) {
-        const bool hi = lane & o;
-#pragma unroll
-        for (int j = 0; j < h; ++j) {
-          const float send = hi ? v[j] : v[j + h];
-          const float keep = hi ? v[j + h] : v[j];
-          v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = unpack2(acc[bb][j]);
+          v[bb * 8 + 2 * j] = f.x;
+          v[bb * 8 + 2 * j + 1] = f.y;
         }
-        if (hi) off += h;
-        held = h;
-      }
-    }
-    __syncthreads();                             // every thread is done with xs
-    if (active) {
+      int off = 0, held = 64;
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        if (j < held) {
-          const int idx = off + j, bb = idx >> 3, c = idx & 7;
-          red[(warp * kProjRows + bb) * r + c0 + c] = v[j];
+      for (int s = 0; s < 5; ++s) {
+        const int h = 32 >> s;                   // values sent (and kept) in this step
+        const int o = tpr << s;
+        if (o < 32) {
+          const bool hi = lane & o;
+#pragma unroll
+          for (int j = 0; j < h; ++j) {
+            const float send = hi ? v[j] : v[j + h];
+            const float keep = hi ? v[j + h] : v[j];
+            v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+          }
+          if (hi) off += h;
+          held = h;
         }
       }
-    }
-    __syncthreads();
-    for (int idx = t; idx < nb * r; idx += kProjThreads) {
-      const int bb = idx / r, k = idx - bb * r;
-      float z = 0.f;
+      if (active) {
 #pragma unroll
-      for (int w = 0; w < kProjWarps; ++w) z += red[(w * kProjRows + bb) * r + k];
-      if (ns == 1) zs[idx] = z;
-      else pa.part[(((size_t)gk * ns + sp) * a.B + b0) * r + idx] = z;
+        for (int j = 0; j < 64; ++j) {
+          if (j < held) {
+            const int idx = off + j, bb = idx >> 3, c = idx & 7;
+            red[(warp * kProjRows + bb) * r + c0 + c] = v[j];
+          }
+        }
+      }
+      __syncthreads();
+      for (int idx = t; idx < nb * r; idx += kProjThreads) {
+        const int bb = idx / r, k = idx - bb * r;
+        float z = 0.f;
+#pragma unroll
+        for (int w = 0; w < kProjWarps; ++w) z += red[(w * kProjRows + bb) * r + k];
+        if (ns == 1) zs[idx] = z;
+        else zc[(size_t)b0 * r + idx] = z;
+      }
+      __syncthreads();
+      if (ns == 1) proj_write_rows<LAT>(pa, 2 * g + kv, b0, nb, zs, lane, warp);
     }
-    __syncthreads();
-    if (ns == 1) proj_write_rows<LAT>(pa, 2 * g + kv, b0, nb, zs, lane, warp);
   }
   if (timed_out) {
     // results are invalid; make sure no copy still writes this CTA's shared memory
@@ -551,38 +675,33 @@ __global__ void __launch_bounds__(kProjThreads, 2) lrkv_project_append_kernel(Pr
     mbar_wait(bar, (copies - 1) & 1, &abort_flag, kWaitNs);
   }
   if (ns > 1) {
-    // the last of the head's 2 nsplit CTAs adds the slices (fixed order) and writes
-    // the head's K and V rows
-    __syncthreads();
-    bool last = false;
-    if (t == 0) {
-      __threadfence();
-      last = atomicAdd(a.header + kProjHeadWord + g, 1u) == 2u * ns - 1u;
-    }
-    if (!__syncthreads_or(last)) return;
-    __threadfence();
-    for (int kvv = 0; kvv < 2; ++kvv) {
-      for (int b0 = 0; b0 < a.B; b0 += kProjRows) {
-        const int nb = min(kProjRows, a.B - b0);
-        __syncthreads();
-        for (int idx = t; idx < nb * r; idx += kProjThreads) {
-          const int bb = idx / r, kk = idx - bb * r;
-          float z = 0.f;
-          for (int q = 0; q < ns; ++q)
-            z += __ldcg(&pa.part[((((size_t)(2 * g + kvv)) * ns + q) * a.B + b0 + bb) * r + kk]);
-          zs[bb * r + kk] = z;
-        }
-        __syncthreads();
-        proj_write_rows<LAT>(pa, 2 * g + kvv, b0, nb, zs, lane, warp);
+    // the ns CTAs of this factor form one cluster: once every partial is in shared
+    // memory, CTA c adds the ns partials of its share of the batch rows (read from the
+    // other CTAs' shared memory, always in rank order) and writes those rows
+    cluster_sync_all();
+    const uint32_t crank = cluster_rank();
+    const int per = (B + ns - 1) / ns;
+    const int blo = min(B, (int)crank * per), bhi = min(B, blo + per);
+    const uint32_t zc_addr = smem_addr(zc);
+    for (int b0 = blo; b0 < bhi; b0 += kProjRows) {
+      const int nb = min(kProjRows, bhi - b0);
+      __syncthreads();
+      for (int idx = t; idx < nb * r; idx += kProjThreads) {
+        const uint32_t off = (uint32_t)(((size_t)b0 * r + idx) * sizeof(float));
+        float z = 0.f;
+        for (int q = 0; q < ns; ++q) z += ld_cluster_f32(zc_addr + off, (uint32_t)q);
+        zs[idx] = z;
       }
+      __syncthreads();
+      proj_write_rows<LAT>(pa, 2 * g + kv, b0, nb, zs, lane, warp);
     }
-    if (t == 0) atomicExch(a.header + kProjHeadWord + g, 0u);
+    cluster_sync_all();   // no CTA leaves while another still reads its partial sums
   }
   // the last writer advances every valid row's length (all writers have read it)
   __syncthreads();
   if (t == 0) {
     __threadfence();
-    const unsigned writers = ns > 1 ? (unsigned)a.Hkv : gridDim.x;
+    const unsigned writers = gridDim.x * gridDim.y;
     const unsigned prev = atomicAdd(a.header + kProjCounter, 1u);
     if (prev == writers - 1) {
       __threadfence();
@@ -641,8 +760,13 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t st) {
 template <int LAT, int IO>
 cudaError_t launch_project_typed(const ProjArgs& a, cudaStream_t st) {
   const int e = IO == LRKV_F32 ? 4 : 2;
-  const int dspan = (a.d_model + a.nsplit - 1) / a.nsplit;
-  const size_t smem = proj_smem_bytes(a.app.r, e, proj_chunk_rows(a.app.r, e, dspan));
+  const int dspan = proj_dspan(a.d_model, a.nsplit);
+  const int cr = proj_chunk_rows(a.app.r, e, dspan);
+  // the largest slice decides (the last slice is shorter, never longer)
+  const bool chunked = std::min(dspan, a.d_model) > cr;
+  const size_t smem = proj_smem_bytes(a.app.B, a.app.r, e, cr,
+                                      proj_batch_block(a.app.B, a.app.r, e, cr, chunked, a.nsplit),
+                                      a.nsplit);
   static size_t configured = 48 * 1024;
   if (smem > configured) {
     cudaError_t err = cudaFuncSetAttribute(lrkv_project_append_kernel<LAT, IO>,
@@ -650,8 +774,21 @@ cudaError_t launch_project_typed(const ProjArgs& a, cudaStream_t st) {
     if (err != cudaSuccess) return err;
     configured = smem;
   }
-  return launch_pdl(lrkv_project_append_kernel<LAT, IO>, dim3(2 * a.app.Hkv, a.nsplit),
-                    dim3(kProjThreads), smem, st, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * a.app.Hkv, a.nsplit);
+  cfg.blockDim = dim3(kProjThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;   // the CTAs of one factor
+  attr[1].val.clusterDim.x = 1;
+  attr[1].val.clusterDim.y = a.nsplit;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, lrkv_project_append_kernel<LAT, IO>, a);
 }
 
 template <int LAT>
@@ -670,15 +807,15 @@ cudaError_t launch_project_append(const ProjArgs& a, cudaStream_t st) {
 }
 
 int project_nsplit(int Hkv, int B, int r, int d_model, int io_bytes, size_t workspace_bytes) {
-  if (Hkv > kProjMaxHeads) return 1;
+  (void)workspace_bytes;   // the partial sums live in the cluster's shared memory
+  // the CTAs of one factor form a cluster and keep every batch row's partial sums
+  if ((size_t)B * r * sizeof(float) > (size_t)kProjClusterBytes) return 1;
   // one wave of two CTAs per SM, or more CTAs if a slice would not fit in shared
-  // memory, each with at least kProjMinSpan rows of the factor
+  // memory; at most one portable cluster, each CTA with at least kProjMinSpan rows
   const int cap = proj_chunk_rows(r, io_bytes, d_model);
   int ns = std::max(std::max(1, 2 * num_sms() / (2 * Hkv)), (d_model + cap - 1) / cap);
+  ns = std::min(ns, kProjMaxCluster);
   ns = std::min(ns, std::max(1, d_model / kProjMinSpan));
-  const size_t per = (size_t)2 * Hkv * B * r * sizeof(float);
-  const size_t room = workspace_bytes > kHeaderBytes ? workspace_bytes - kHeaderBytes : 0;
-  ns = (int)std::min<size_t>((size_t)ns, room / per);
   return std::max(1, ns);
 }
 

@@ -299,7 +299,7 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
       int ct = (int)((a.chunk_hint * tiles + full - 1) / full);
       ct = max(a.chunk / kT, min(ct, a.chunk_hint));
       chunk = ct * kT;
-      total_units = ((tiles_max + ct - 1) / ct) * BH;
+      total_units = total_splits(a.n_visual, a.max_seqlen, chunk) * BH;
       if (blockIdx.x == 0 && lane == 0) atomicExch(a.header + kChunkWord, (unsigned)chunk);
     }
     uint32_t tile_seq = 0;
@@ -311,15 +311,14 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
       if (leader) u = (int)atomicAdd(a.header + kWorkCounter, 1u);
       u = __shfl_sync(0xffffffffu, u, 0);
       const bool term = u >= total_units;
-      int b = 0, g = 0, s = 0, t0 = 0, t1 = 0;
+      int b = 0, g = 0, s = 0, t0 = 0, t1 = 0, fset = 0;
       if (!term) {
         s = u / BH;
         const int rem = u - s * BH;
         b = rem / a.Hkv;
         g = rem - b * a.Hkv;
         const int L = checked_len_tc(a, b);
-        t0 = s * chunk;
-        t1 = min(L, t0 + chunk);
+        fset = split_range(s, L, a.n_visual, a.max_seqlen, chunk, &t0, &t1);
         if (t0 >= t1) continue;  // empty split: nothing to do, the merge skips it
       }
       const int us = unit_seq % kUR;
@@ -347,8 +346,10 @@ __global__ void __launch_bounds__(Roles<LAT>::kThreads, 2)
         const uint32_t sbv = sbk + fac_bytes;
         mbar_arrive_expect_tx(bar(BAR_BQFULL + bx), 2u * fac_bytes + q_bytes);
         for (int blk = 0; blk < 2; ++blk) {
-          tma_load_2d(sbk + (uint32_t)blk * (uint32_t)r * 128u, &p.tm_bk, bar(BAR_BQFULL + bx), blk * 64, g * r);
-          tma_load_2d(sbv + (uint32_t)blk * (uint32_t)r * 128u, &p.tm_bv, bar(BAR_BQFULL + bx), blk * 64, g * r);
+          // factor rows of this head in the unit's set (visual / text when separated)
+          const int frow = (fset * a.Hkv + g) * r;
+          tma_load_2d(sbk + (uint32_t)blk * (uint32_t)r * 128u, &p.tm_bk, bar(BAR_BQFULL + bx), blk * 64, frow);
+          tma_load_2d(sbv + (uint32_t)blk * (uint32_t)r * 128u, &p.tm_bv, bar(BAR_BQFULL + bx), blk * 64, frow);
         }
         const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q) +
                                   ((size_t)b * a.Hq + (size_t)g * G) * kD;
@@ -1162,10 +1163,9 @@ cudaError_t launch_split_tc(const SplitArgs& a, const Plan& plan, cudaStream_t s
     ok &= make_tmap_vec_f32(&prm.tm_sk, a.SK, rows);
     ok &= make_tmap_vec_f32(&prm.tm_sv, a.SV, rows);
   }
-  ok &= make_tmap_2d(&prm.tm_bk, a.BK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD,
-                     (uint64_t)a.Hkv * a.r, 64, a.r, 128);
-  ok &= make_tmap_2d(&prm.tm_bv, a.BV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD,
-                     (uint64_t)a.Hkv * a.r, 64, a.r, 128);
+  const uint64_t fac_rows = (uint64_t)(a.n_visual > 0 ? 2 : 1) * a.Hkv * a.r;
+  ok &= make_tmap_2d(&prm.tm_bk, a.BK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, fac_rows, 64, a.r, 128);
+  ok &= make_tmap_2d(&prm.tm_bv, a.BV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, fac_rows, 64, a.r, 128);
   if (!ok) return cudaErrorInvalidValue;
   prm.a = a;
   prm.total_units = a.S * a.B * a.Hkv;

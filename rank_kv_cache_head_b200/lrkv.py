@@ -40,7 +40,7 @@ class LrkvError(RuntimeError):
 class Dims(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "batch", "n_q_heads", "n_kv_heads", "d_head", "rank", "max_seq", "max_seqlen",
-        "io_dtype", "latent_dtype", "num_splits", "algo")]
+        "io_dtype", "latent_dtype", "num_splits", "algo", "n_visual")]
 
     def __repr__(self):
         return "Dims(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -94,11 +94,14 @@ def strerror(code: int) -> str:
 
 
 def make_dims(batch, n_q_heads, n_kv_heads, d_head, rank, max_seq, max_seqlen,
-              io_dtype="bf16", latent_dtype="bf16", num_splits=0, algo="auto") -> Dims:
+              io_dtype="bf16", latent_dtype="bf16", num_splits=0, algo="auto",
+              n_visual=0) -> Dims:
+    """n_visual > 0: modality-separated factors, BK/BV [2][Hkv][r][d] (visual set for
+    positions < n_visual, text set after)."""
     return Dims(batch, n_q_heads, n_kv_heads, d_head, rank, max_seq, max_seqlen,
                 DTYPE_CODE[io_dtype] if isinstance(io_dtype, str) else io_dtype,
                 DTYPE_CODE[latent_dtype] if isinstance(latent_dtype, str) else latent_dtype,
-                num_splits, ALGO_CODE[algo] if isinstance(algo, str) else algo)
+                num_splits, ALGO_CODE[algo] if isinstance(algo, str) else algo, n_visual)
 
 
 def plan(dims: Dims) -> dict:
@@ -152,7 +155,7 @@ def _shapes(d: Dims):
         "q": (d.batch * d.n_q_heads * d.d_head, (io,)),
         "Z": (d.batch * d.n_kv_heads * d.max_seq * d.rank, _LATENT_TORCH_OK[d.latent_dtype]),
         "S": (d.batch * d.n_kv_heads * d.max_seq, (torch.float32,)),
-        "B": (d.n_kv_heads * d.rank * d.d_head, (io,)),
+        "B": ((2 if d.n_visual > 0 else 1) * d.n_kv_heads * d.rank * d.d_head, (io,)),
         "znew": (d.batch * d.n_kv_heads * d.rank, (io,)),
         "seq": (d.batch, (torch.int32,)),
         "lse": (d.batch * d.n_q_heads, (torch.float32,)),

@@ -22,13 +22,13 @@ import numpy as np
 _BYTES = {"f32": 4, "bf16": 2, "i8": 1, "e4m3": 1}
 
 
-def step_bytes(wl, seqlens) -> dict:
+def step_bytes(wl, seqlens, factor_sets: int = 1) -> dict:
     tok_heads = int(np.sum(np.asarray(seqlens, np.int64))) * wl.n_kv_heads
     quant = wl.latent_dtype in ("i8", "e4m3")
     latent = tok_heads * 2 * wl.rank * _BYTES[wl.latent_dtype]
     scales = tok_heads * 2 * 4 if quant else 0
     io = _BYTES[wl.io_dtype]
-    factors = 2 * wl.n_kv_heads * wl.rank * wl.d_head * io
+    factors = factor_sets * 2 * wl.n_kv_heads * wl.rank * wl.d_head * io
     q = wl.batch * wl.n_q_heads * wl.d_head * io
     out = q
     total = latent + scales + factors + q + out

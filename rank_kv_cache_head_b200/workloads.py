@@ -205,6 +205,22 @@ def make_inputs(wl: Workload, capacity: Optional[int] = None, poison: Optional[s
     return out
 
 
+def with_text_factors(wl: Workload, inputs: dict) -> dict:
+    """Modality-separated factors: a copy of ``inputs`` whose BK/BV are [2][Hkv][r][d],
+    the workload's own factors (the visual set) followed by a second set drawn the same
+    way from another seed (the text set)."""
+    rng = np.random.default_rng(np.random.PCG64(wl.seed + 1000))
+    sig = sigmas(wl)
+    io_t = _TORCH_DTYPE[wl.io_dtype]
+    out = dict(inputs)
+    for k in ("BK", "BV"):
+        f = np.stack([sig[:, None] * _orthonormal_rows(rng, wl.rank, wl.d_head)
+                      for _ in range(wl.n_kv_heads)])
+        text = torch.from_numpy(np.ascontiguousarray(f)).to(io_t)
+        out[k] = torch.stack([inputs[k], text]).contiguous()
+    return out
+
+
 def make_append_rows(wl: Workload, step: int = 0) -> dict:
     """New latent rows for one append: zk_new, zv_new [B][Hkv][r] in the io dtype."""
     rng = np.random.default_rng(np.random.PCG64(wl.seed * 7919 + 13 + step))

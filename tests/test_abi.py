@@ -29,7 +29,7 @@ def test_library_exports_every_declared_function():
     L = lrkv.lib()
     missing = [n for n in declared_functions() if not hasattr(L, n)]
     assert not missing, missing
-    assert lrkv.version() == 1
+    assert lrkv.version() == 2
 
 
 def test_strerror_codes():
@@ -61,6 +61,9 @@ def _plan_rc(d):
     (dict(io_dtype="bf16", latent_dtype="f32"), -2),
     (dict(latent_dtype="i8", rank=8), -3),
     (dict(num_splits=-1), -1),
+    (dict(n_visual=8), -1),             # modality boundary not a multiple of 16
+    (dict(n_visual=-16), -1),
+    (dict(n_visual=4096), -1),          # past the capacity
 ])
 def test_invalid_dims_rejected(kw, code):
     assert _plan_rc(_dims(**kw)) == code

@@ -35,6 +35,15 @@ SMALL = {
                                               seq_len=400, seed=17),
     "d64-bf16": WORKLOADS["vlm7b-bf16"].scaled(batch=2, n_q_heads=4, n_kv_heads=2, d_head=64,
                                                rank=16, seq_len=300, seed=18),
+    # the remaining group sizes and latent formats of the tensor-core kernel
+    "g8-rank48": WORKLOADS["vlm7b-bf16"].scaled(batch=3, n_q_heads=16, n_kv_heads=2, rank=48,
+                                                seq_len=555, seed=19),
+    "quant-i8-g1-rank64": WORKLOADS["quant-i8"].scaled(batch=2, n_q_heads=2, n_kv_heads=2,
+                                                       rank=64, seq_len=640, seed=20),
+    "quant-e4m3-g16": WORKLOADS["quant-e4m3"].scaled(batch=2, n_q_heads=32, n_kv_heads=2,
+                                                     seq_len=132, seed=21),
+    "quant-i8-g2-rank128": WORKLOADS["quant-i8"].scaled(batch=2, n_q_heads=4, n_kv_heads=2,
+                                                        rank=128, seq_len=300, seed=22),
 }
 
 

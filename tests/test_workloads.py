@@ -31,6 +31,22 @@ def test_factor_rows_are_orthonormal_times_sigma():
     assert np.allclose(gram, np.diag(sig ** 2), atol=1e-6)
 
 
+def test_text_factor_set_is_a_second_draw_of_the_same_recipe():
+    from rank_kv_cache_head_b200.workloads import with_text_factors
+    wl = WORKLOADS["vlm7b-bf16"].scaled(batch=1, seq_len=64, n_q_heads=2, n_kv_heads=2,
+                                        io_dtype="f32", latent_dtype="f32")
+    x = make_inputs(wl)
+    m = with_text_factors(wl, x)
+    assert m["BK"].shape == (2, 2, wl.rank, wl.d_head) and m["BK"].is_contiguous()
+    assert torch.equal(m["BK"][0], x["BK"]) and torch.equal(m["BV"][0], x["BV"])
+    assert not torch.equal(m["BK"][1], x["BK"]) and not torch.equal(m["BK"][1], m["BV"][1])
+    sig = sigmas(wl)
+    for k in ("BK", "BV"):
+        T = m[k][1][1].double().numpy()
+        assert np.allclose(T @ T.T, np.diag(sig ** 2), atol=1e-6)
+    assert m["ZK"] is x["ZK"]
+
+
 def test_outlier_positions_scaled():
     wl = WORKLOADS["longvideo-bf16"].scaled(batch=1, seq_len=1000, io_dtype="f32",
                                             latent_dtype="f32")
