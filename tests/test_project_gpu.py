@@ -24,7 +24,7 @@ def _decode(bits, lat):
     return orc.decode_stored(bits, lat)
 
 
-@pytest.mark.parametrize("ws_bytes", [256, 4 << 20])   # header only: no split; room: split
+@pytest.mark.parametrize("ws_bytes", [256, 4 << 20])   # only the header is used: same result
 @pytest.mark.parametrize("io,lat,r,D,B", [("f32", "f32", 32, 300, 3), ("bf16", "bf16", 32, 300, 3),
                                           ("bf16", "bf16", 48, 1000, 3), ("bf16", "i8", 32, 520, 3),
                                           ("bf16", "e4m3", 64, 2304, 3),
