@@ -384,6 +384,11 @@ constexpr int kProjMinSpan = 64;          // fewest hidden-size rows a CTA takes
 constexpr int kProjMaxCluster = 8;        // CTAs sharing one factor: one portable cluster
 constexpr int kProjClusterBytes = 32 * 1024;  // a CTA's partial sums [B][r] must fit this
 
+// batch rows per block of the grid's z dimension (a multiple of 8)
+__host__ __device__ inline int proj_batch_rows(int B, int nbz) {
+  return ((B + nbz - 1) / nbz + 7) / 8 * 8;
+}
+
 // hidden-size rows per CTA: a multiple of 8, so 16-byte loads of x stay aligned
 __host__ __device__ inline int proj_dspan(int D, int ns) { return ((D + ns - 1) / ns + 7) / 8 * 8; }
 
@@ -536,8 +541,11 @@ __global__ void __launch_bounds__(kProjThreads, 2) lrkv_project_append_kernel(Pr
   extern __shared__ __align__(16) unsigned char proj_smem[];
   __shared__ int abort_flag;
   const AppendArgs& a = pa.app;
-  const int r = a.r, B = a.B;
+  const int r = a.r;
   const int gk = blockIdx.x, g = gk >> 1, kv = gk & 1, sp = blockIdx.y, ns = pa.nsplit;
+  // this CTA's block of batch rows [Blo, Blo + B) (blockIdx.z; may be empty)
+  const int Bb = proj_batch_rows(a.B, gridDim.z);
+  const int Blo = min(a.B, (int)blockIdx.z * Bb), B = min(a.B, Blo + Bb) - Blo;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int D = pa.d_model;
   const int dspan = proj_dspan(D, ns);
@@ -547,14 +555,14 @@ __global__ void __launch_bounds__(kProjThreads, 2) lrkv_project_append_kernel(Pr
   const bool resident = nchunks == 1;
   // the launch's shared memory is sized for the longest slice, so the block of batch
   // rows depends on that slice, not on this CTA's (the last one may be shorter)
-  const int bblk = proj_batch_block(B, r, E, cr, min(dspan, D) > cr, ns);
+  const int bblk = proj_batch_block(Bb, r, E, cr, min(dspan, D) > cr, ns);
   const bool vec = (D % 8 == 0) && ((reinterpret_cast<uintptr_t>(pa.x) & 15) == 0);
   const uint32_t bar = smem_addr(proj_smem);
   char* As = reinterpret_cast<char*>(proj_smem + 16);              // [row][r] as in A
   float* xs = reinterpret_cast<float*>(As + (size_t)cr * r * E);   // [batch row][row]
   float* red = xs + (size_t)bblk * cr;                             // [warp][batch row][col]
   float* zs = red + kProjWarps * kProjRows * r;                    // [batch row][col]
-  float* zc = zs + kProjRows * r;              // ns > 1: this CTA's partial sums [B][r]
+  float* zc = zs + kProjRows * r;              // ns > 1: this CTA's partial sums [Bb][r]
   const char* A = static_cast<const char*>(kv ? pa.AV : pa.AK) + (size_t)g * D * r * E;
   const size_t row_bytes = (size_t)r * E;
   if (t == 0) {
@@ -582,8 +590,8 @@ __global__ void __launch_bounds__(kProjThreads, 2) lrkv_project_append_kernel(Pr
   const int nslots = kProjWarps * spw, slot = warp * spw + lane / tpr;
   const bool active = c0 < r;
 
-  for (int blk0 = 0; blk0 < B; blk0 += bblk) {
-    const int nblk = min(bblk, B - blk0);
+  for (int blk0 = Blo; blk0 < Blo + B; blk0 += bblk) {
+    const int nblk = min(bblk, Blo + B - blk0);
     for (int g8 = 0; g8 < nblk; g8 += kProjRows) {
       const int b0 = blk0 + g8, nb = min(kProjRows, nblk - g8);
       uint64_t acc[kProjRows][4];
@@ -662,7 +670,7 @@ __global__ void __launch_bounds__(kProjThreads, 2) lrkv_project_append_kernel(Pr
 #pragma unroll
         for (int w = 0; w < kProjWarps; ++w) z += red[(w * kProjRows + bb) * r + k];
         if (ns == 1) zs[idx] = z;
-        else zc[(size_t)b0 * r + idx] = z;
+        else zc[(size_t)(b0 - Blo) * r + idx] = z;
       }
       __syncthreads();
       if (ns == 1) proj_write_rows<LAT>(pa, 2 * g + kv, b0, nb, zs, lane, warp);
@@ -681,13 +689,13 @@ __global__ void __launch_bounds__(kProjThreads, 2) lrkv_project_append_kernel(Pr
     cluster_sync_all();
     const uint32_t crank = cluster_rank();
     const int per = (B + ns - 1) / ns;
-    const int blo = min(B, (int)crank * per), bhi = min(B, blo + per);
+    const int blo = min(B, (int)crank * per), bhi = min(B, blo + per);   // within the block
     const uint32_t zc_addr = smem_addr(zc);
-    for (int b0 = blo; b0 < bhi; b0 += kProjRows) {
-      const int nb = min(kProjRows, bhi - b0);
+    for (int l0 = blo; l0 < bhi; l0 += kProjRows) {
+      const int nb = min(kProjRows, bhi - l0), b0 = Blo + l0;
       __syncthreads();
       for (int idx = t; idx < nb * r; idx += kProjThreads) {
-        const uint32_t off = (uint32_t)(((size_t)b0 * r + idx) * sizeof(float));
+        const uint32_t off = (uint32_t)(((size_t)l0 * r + idx) * sizeof(float));
         float z = 0.f;
         for (int q = 0; q < ns; ++q) z += ld_cluster_f32(zc_addr + off, (uint32_t)q);
         zs[idx] = z;
@@ -701,7 +709,7 @@ __global__ void __launch_bounds__(kProjThreads, 2) lrkv_project_append_kernel(Pr
   __syncthreads();
   if (t == 0) {
     __threadfence();
-    const unsigned writers = gridDim.x * gridDim.y;
+    const unsigned writers = gridDim.x * gridDim.y * gridDim.z;
     const unsigned prev = atomicAdd(a.header + kProjCounter, 1u);
     if (prev == writers - 1) {
       __threadfence();
@@ -764,8 +772,13 @@ cudaError_t launch_project_typed(const ProjArgs& a, cudaStream_t st) {
   const int cr = proj_chunk_rows(a.app.r, e, dspan);
   // the largest slice decides (the last slice is shorter, never longer)
   const bool chunked = std::min(dspan, a.d_model) > cr;
-  const size_t smem = proj_smem_bytes(a.app.B, a.app.r, e, cr,
-                                      proj_batch_block(a.app.B, a.app.r, e, cr, chunked, a.nsplit),
+  // batch blocks over the grid's z dimension while the (factor, slice) CTAs leave SMs
+  // idle: about two CTAs per SM in all, each with at least 8 rows
+  const int ctas = 2 * a.app.Hkv * a.nsplit;
+  const int nbz = std::max(1, std::min((a.app.B + 7) / 8, 2 * num_sms() / ctas));
+  const int Bb = proj_batch_rows(a.app.B, nbz);
+  const size_t smem = proj_smem_bytes(Bb, a.app.r, e, cr,
+                                      proj_batch_block(Bb, a.app.r, e, cr, chunked, a.nsplit),
                                       a.nsplit);
   static size_t configured = 48 * 1024;
   if (smem > configured) {
@@ -775,7 +788,7 @@ cudaError_t launch_project_typed(const ProjArgs& a, cudaStream_t st) {
     configured = smem;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * a.app.Hkv, a.nsplit);
+  cfg.gridDim = dim3(2 * a.app.Hkv, a.nsplit, nbz);
   cfg.blockDim = dim3(kProjThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
