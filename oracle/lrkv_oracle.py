@@ -195,6 +195,67 @@ def decode_attention(q, ZK, ZV, BK, BV, seqlens, ZK_scale=None, ZV_scale=None,
     return out, lse
 
 
+def decode_attention_adaptive(q, ZK, ZV, BK, BV, seqlens, importance, tau: float, r_low: int,
+                              beta: float, ZK_scale=None, ZV_scale=None, n_visual: int = 0):
+    """Attention-aware partial decompression ("AttentionPack", Metodologia 2.B): tokens
+    whose tracked importance is high are rebuilt at the full rank, the others with the
+    leading r_low rank components only (the factor rows are ordered by singular value,
+    so a prefix is the best rank-r_low part); the accumulated attention is tracked with
+    a moving average.
+
+    Readings: importance is kept per (batch row, KV head, token) in ``importance``
+    [B][Hkv][L_cap] (fp32 values); a token is important when importance >= tau (the
+    comparison of the stored fp32 values); the reduced rank applies to both the key and
+    the value row; a token's attention mass is its softmax weight summed over the G query
+    heads of the group, and the moving average is imp <- beta * imp + (1 - beta) * mass
+    for the attended positions (the others are left unchanged).
+
+    Returns out [B][Hq][d], lse [B][Hq], mass [B][Hkv][L_cap] (0 past the length) and
+    the updated importance [B][Hkv][L_cap] (float64)."""
+    q = np.asarray(q, np.float64)
+    B, Hq, d = q.shape
+    Hkv, Lc, r = ZK.shape[1], ZK.shape[2], ZK.shape[3]
+    G = Hq // Hkv
+    imp = np.asarray(importance, np.float64)
+    out = np.zeros((B, Hq, d))
+    lse = np.full((B, Hq), -np.inf)
+    mass = np.zeros((B, Hkv, Lc))
+    for b in range(B):
+        Lb = int(seqlens[b])
+        if Lb == 0:
+            continue
+        for g in range(Hkv):
+            sk = None if ZK_scale is None else ZK_scale[b, g, :Lb]
+            sv = None if ZV_scale is None else ZV_scale[b, g, :Lb]
+            Zk = dequantise(np.asarray(ZK[b, g, :Lb, :], np.float64), sk)
+            Zv = dequantise(np.asarray(ZV[b, g, :Lb, :], np.float64), sv)
+            # reduced-rank tokens keep only their leading r_low latent components
+            low = imp[b, g, :Lb] < tau
+            Zk[low, r_low:] = 0.0
+            Zv[low, r_low:] = 0.0
+            K = np.zeros((Lb, d))
+            V = np.zeros((Lb, d))
+            for t in range(Lb):
+                m = 0 if (n_visual == 0 or t < n_visual) else 1
+                fk = BK[m][g] if n_visual else BK[g]
+                fv = BV[m][g] if n_visual else BV[g]
+                K[t] = Zk[t] @ np.asarray(fk, np.float64)
+                V[t] = Zv[t] @ np.asarray(fv, np.float64)
+            for h in range(g * G, (g + 1) * G):
+                s = (K @ q[b, h]) / math.sqrt(d)
+                mx = s.max()
+                e = np.exp(s - mx)
+                l = e.sum()
+                out[b, h] = (e / l) @ V
+                lse[b, h] = mx + math.log(l)
+                mass[b, g, :Lb] += e / l
+    new_imp = imp.copy()
+    for b in range(B):
+        Lb = int(seqlens[b])
+        new_imp[b, :, :Lb] = beta * imp[b, :, :Lb] + (1.0 - beta) * mass[b, :, :Lb]
+    return out, lse, mass, new_imp
+
+
 def decode_attention_reassociated(q, ZK, ZV, BK, BV, seqlens, ZK_scale=None, ZV_scale=None):
     """The same attention computed without rebuilding K, V: scores as
     (q B_K^T) Z_K^T and output as (p Z_V) B_V. Exactly equal in real arithmetic;
