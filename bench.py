@@ -67,6 +67,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--projection-dmodel", type=int, default=4096,
                     help="also time lrkv_project_append with this hidden size (0: skip)")
+    ap.add_argument("--adaptive-rlow", type=int, default=0, metavar="R",
+                    help="also time the attention-aware partial decompression with tokens "
+                         "below the importance threshold rebuilt at rank R (0: skip)")
     ap.add_argument("--n-visual", type=int, default=0, metavar="P",
                     help="modality-separated factors: positions < P use a visual factor "
                          "set, the rest a text set (0: one set, the default)")
@@ -322,6 +325,69 @@ def measure_projection(wl, dev, d_model: int):
             "factors": f"rotated over {n_a} copies ({n_a * a_bytes / 1e6:.0f} MB)"}
 
 
+def measure_adaptive(wl, dev, r_low: int, tau: float = 0.5, beta: float = 0.9):
+    """Time lrkv_decode_attn_adaptive (attention-aware partial decompression, CUDA-core
+    kernel) on this workload beside the plain CUDA-core decode of the same cache: about
+    half of the tokens (importance drawn uniform in [0, 1], tau 0.5) are rebuilt at rank
+    r_low. Each timed call also updates the importance. Returns a dict for the JSON line."""
+    target = seqlens_for(wl)
+    cap = ((int(target.max()) + 7) // 8) * 8
+    x = make_inputs(wl, capacity=cap, seqlens=target)
+    d = {k: (None if v is None else v.to(dev)) for k, v in x.items()}
+    dims = lrkv.make_dims(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.d_head, wl.rank, cap,
+                          int(target.max()), wl.io_dtype, wl.latent_dtype, 0, "simt")
+    g = torch.Generator(device="cpu").manual_seed(wl.seed + 77)
+    imp = torch.rand(wl.batch, wl.n_kv_heads, cap, generator=g).to(dev)
+    low_frac = float((imp.cpu()[..., :int(target.max())] < tau).float().mean())
+    scores = torch.empty(wl.batch, wl.n_q_heads, cap, dtype=torch.float32, device=dev)
+    out = torch.empty_like(d["q"])
+    lse = torch.empty(wl.batch, wl.n_q_heads, dtype=torch.float32, device=dev)
+    ws = lrkv.new_workspace(dims, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    adaptive = lambda: lrkv.decode_attn_adaptive(dims, d["q"], d["ZK"], d["ZV"], d["ZK_scale"],
+                                                 d["ZV_scale"], d["BK"], d["BV"], d["seqlens"], imp,
+                                                 tau, r_low, beta, scores, out, lse, ws, stream=stream)
+    plain = lambda: lrkv.decode_attn(dims, d["q"], d["ZK"], d["ZV"], d["ZK_scale"], d["ZV_scale"],
+                                     d["BK"], d["BV"], d["seqlens"], out, ws, lse_out=lse,
+                                     stream=stream)
+    per_graph, replays = 10, 3
+
+    def time_it(fn):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
+            stream.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                for _ in range(per_graph):
+                    fn()
+            graph.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(replays):
+                graph.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1e3 / (per_graph * replays)
+
+    us_plain = time_it(plain)
+    us_adapt = time_it(adaptive)
+    st = lrkv.read_status(ws)
+    if st:
+        raise RuntimeError(f"device status {st} after the adaptive timing")
+    sb = step_bytes(wl, target)
+    lat = sb["latent"] + sb["scales"]
+    peak, kind = peaks()
+    return {"kernel": "CUDA-core split (simt) + merge + attention-mass moving average",
+            "r_low": r_low, "rank": wl.rank, "tau": tau, "beta": beta,
+            "low_rank_token_fraction": low_frac,
+            "reconstruction_flops_fraction": low_frac * r_low / wl.rank + (1 - low_frac),
+            "us_per_call": us_adapt, "simt_plain_us_per_call": us_plain,
+            "latent_GBs": lat / (us_adapt * 1e-6) / 1e9, "peak_GBs": peak, "peak_kind": kind,
+            "frac": lat / (us_adapt * 1e-6) / 1e9 / peak,
+            "launches": f"CUDA graph of {per_graph} calls, one cache copy"}
+
+
 def run_ours(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -524,6 +590,8 @@ def run_ours(args, rank, world, local):
     }
     if args.projection_dmodel > 0:
         line["project_append"] = measure_projection(wl, dev, args.projection_dmodel)
+    if rank == 0 and args.adaptive_rlow > 0:
+        line["adaptive"] = measure_adaptive(wl, dev, args.adaptive_rlow)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         per_unit, n, lb, spent = oracle_sample(wl, inputs, args.cpu_seconds, n_visual=args.n_visual)
         cores = blas_threads()

@@ -227,8 +227,9 @@ def decode_attention_adaptive(q, ZK, ZV, BK, BV, seqlens, importance, tau: float
         for g in range(Hkv):
             sk = None if ZK_scale is None else ZK_scale[b, g, :Lb]
             sv = None if ZV_scale is None else ZV_scale[b, g, :Lb]
-            Zk = dequantise(np.asarray(ZK[b, g, :Lb, :], np.float64), sk)
-            Zv = dequantise(np.asarray(ZV[b, g, :Lb, :], np.float64), sv)
+            # copies: the reduced-rank rows are edited below, the inputs stay as given
+            Zk = np.array(dequantise(np.asarray(ZK[b, g, :Lb, :], np.float64), sk))
+            Zv = np.array(dequantise(np.asarray(ZV[b, g, :Lb, :], np.float64), sv))
             # reduced-rank tokens keep only their leading r_low latent components
             low = imp[b, g, :Lb] < tau
             Zk[low, r_low:] = 0.0

@@ -12,7 +12,9 @@
 #include <tuple>
 #include <vector>
 
+#include "lrkv_adaptive_internal.h"
 #include "lrkv_internal.h"
+#include "lrkv_adaptive.h"
 
 namespace lrkv {
 
@@ -229,14 +231,19 @@ int lrkv_decode_attn(const lrkv_dims* dims, const void* q, const void* ZK, const
                                 lse_out, workspace, workspace_bytes, stream, nullptr, nullptr);
 }
 
-int lrkv_decode_attn_timed(const lrkv_dims* dims, const void* q, const void* ZK,
-                           const void* ZV, const float* ZK_scale, const float* ZV_scale,
-                           const void* BK, const void* BV, const int32_t* seqlens, void* out,
-                           float* lse_out, void* workspace, size_t workspace_bytes,
-                           void* stream, void* ev_split_begin, void* ev_split_end) {
+// The decode attention call behind every entry point. ad != nullptr: the attention-
+// aware partial decompression (CUDA-core kernel with a per-token rank, then the
+// moving average of the attention mass after the merge).
+static int decode_impl(const lrkv_dims* dims, const void* q, const void* ZK, const void* ZV,
+                       const float* ZK_scale, const float* ZV_scale, const void* BK,
+                       const void* BV, const int32_t* seqlens, void* out, float* lse_out,
+                       void* workspace, size_t workspace_bytes, void* stream,
+                       void* ev_split_begin, void* ev_split_end, const AdaptArgs* ad,
+                       float beta) {
   Plan p;
   int rc = make_plan(dims, &p);
   if (rc) return rc;
+  if (ad && p.algo != LRKV_ALGO_SIMT) return LRKV_ERR_UNSUPPORTED;
   const bool quant = dims->latent_dtype == LRKV_I8 || dims->latent_dtype == LRKV_E4M3;
   if (!q || !ZK || !ZV || !BK || !BV || !seqlens || !out || !workspace) return LRKV_ERR_ARG;
   if (quant != (ZK_scale != nullptr) || quant != (ZV_scale != nullptr)) return LRKV_ERR_ARG;
@@ -292,8 +299,9 @@ int lrkv_decode_attn_timed(const lrkv_dims* dims, const void* q, const void* ZK,
     a.device_chunk = p.device_chunk;
   }
   record_event(ev_split_begin, st);
-  cudaError_t e = (p.algo == LRKV_ALGO_TCGEN05) ? launch_split_tc(a, p, st)
-                                                : launch_split_simt(a, p, st);
+  cudaError_t e = ad ? launch_split_simt_adaptive(a, *ad, p, st)
+                     : (p.algo == LRKV_ALGO_TCGEN05) ? launch_split_tc(a, p, st)
+                                                     : launch_split_simt(a, p, st);
   if (e != cudaSuccess) return LRKV_ERR_LAUNCH;
   record_event(ev_split_end, st);
 
@@ -315,7 +323,54 @@ int lrkv_decode_attn_timed(const lrkv_dims* dims, const void* q, const void* ZK,
   m.io_dtype = a.io_dtype;
   m.device_chunk = a.device_chunk;
   if (launch_merge(m, st) != cudaSuccess) return LRKV_ERR_LAUNCH;
+  if (ad) {
+    MassArgs ma;
+    ma.scores = ad->scores;
+    ma.lse = lse_out;
+    ma.imp = const_cast<float*>(ad->imp);
+    ma.seqlens = seqlens;
+    ma.header = header;
+    ma.B = a.B;
+    ma.Hq = a.Hq;
+    ma.Hkv = a.Hkv;
+    ma.Lcap = a.Lcap;
+    ma.max_seqlen = a.max_seqlen;
+    ma.beta = beta;
+    if (launch_mass_ema(ma, st) != cudaSuccess) return LRKV_ERR_LAUNCH;
+  }
   return LRKV_OK;
+}
+
+int lrkv_decode_attn_timed(const lrkv_dims* dims, const void* q, const void* ZK,
+                           const void* ZV, const float* ZK_scale, const float* ZV_scale,
+                           const void* BK, const void* BV, const int32_t* seqlens, void* out,
+                           float* lse_out, void* workspace, size_t workspace_bytes,
+                           void* stream, void* ev_split_begin, void* ev_split_end) {
+  return decode_impl(dims, q, ZK, ZV, ZK_scale, ZV_scale, BK, BV, seqlens, out, lse_out,
+                     workspace, workspace_bytes, stream, ev_split_begin, ev_split_end, nullptr,
+                     0.f);
+}
+
+int lrkv_decode_attn_adaptive(const lrkv_dims* dims, const void* q, const void* ZK,
+                              const void* ZV, const float* ZK_scale, const float* ZV_scale,
+                              const void* BK, const void* BV, const int32_t* seqlens,
+                              float* importance, float tau, int32_t r_low, float beta,
+                              float* scores, void* out, float* lse_out, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (dims->algo == LRKV_ALGO_TCGEN05) return LRKV_ERR_UNSUPPORTED;
+  if (!importance || !scores || !lse_out) return LRKV_ERR_ARG;
+  if (r_low < 1 || r_low > dims->rank || !(beta >= 0.f && beta <= 1.f)) return LRKV_ERR_ARG;
+  lrkv_dims d = *dims;
+  d.algo = LRKV_ALGO_SIMT;   // the per-token rank is a loop bound of the CUDA-core kernel
+  AdaptArgs ad;
+  ad.imp = importance;
+  ad.tau = tau;
+  ad.r_low = r_low;
+  ad.scores = scores;
+  return decode_impl(&d, q, ZK, ZV, ZK_scale, ZV_scale, BK, BV, seqlens, out, lse_out,
+                     workspace, workspace_bytes, stream, nullptr, nullptr, &ad, beta);
 }
 
 int lrkv_append(const lrkv_dims* dims, const void* zk_new, const void* zv_new, void* ZK,

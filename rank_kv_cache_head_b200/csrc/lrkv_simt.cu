@@ -15,6 +15,7 @@
 #include <cuda_fp8.h>
 #include <math_constants.h>
 
+#include "lrkv_adaptive_internal.h"
 #include "lrkv_internal.h"
 #include "lrkv_sm100.cuh"
 
@@ -63,7 +64,12 @@ __device__ __forceinline__ int checked_len(const int32_t* seqlens, int b, int Lc
 // heads of the group. Tiles of 32 tokens: latents -> smem (dequantised), rebuild the
 // K tile = Z_K B_K, scores for the G heads, rebuild the V tile = Z_V B_V, online
 // softmax, accumulate P V. fp32 throughout.
-__global__ void __launch_bounds__(kSimtThreads) lrkv_split_simt(SplitArgs a) {
+// ADAPT: attention-aware partial decompression. A token whose importance is below
+// ad.tau is rebuilt from its first ad.r_low latent components (the loop bound of the
+// reconstruction), and the scores of the attended tokens are kept for the moving
+// average of the attention mass.
+template <bool ADAPT>
+__device__ __forceinline__ void split_simt_body(const SplitArgs& a, const AdaptArgs& ad) {
   extern __shared__ float sm[];
   griddep_wait();
   griddep_launch_dependents();
@@ -87,6 +93,7 @@ __global__ void __launch_bounds__(kSimtThreads) lrkv_split_simt(SplitArgs a) {
   float* ms = acc + G * d;        // [G] running max (log2 units)
   float* ls = ms + G;             // [G] running sum
   float* al = ls + G;             // [G] rescale factor of the current tile
+  int* rk = reinterpret_cast<int*>(al + G);   // [T] rank of each token of the tile
 
   const size_t fac_base = ((size_t)fset * a.Hkv + g) * r * d;   // factor set, then head
   for (int i = tid; i < r * d; i += kSimtThreads) {
@@ -124,12 +131,17 @@ __global__ void __launch_bounds__(kSimtThreads) lrkv_split_simt(SplitArgs a) {
       zk[i] = vk;
       zv[i] = vv;
     }
+    if (ADAPT) {
+      for (int t = tid; t < T; t += kSimtThreads)
+        rk[t] = (t < n && ad.imp[row_base + t0 + t] >= ad.tau) ? r : ad.r_low;
+    }
     __syncthreads();
-    // rebuilt key tile K = Z_K B_K
+    // rebuilt key tile K = Z_K B_K (a warp shares one token, so the rank is uniform)
     for (int i = tid; i < T * d; i += kSimtThreads) {
       const int t = i / d, c = i - t * d;
+      const int kr = ADAPT ? rk[t] : r;
       float sum = 0.f;
-      for (int k = 0; k < r; ++k) sum = fmaf(zk[t * r + k], bk[k * d + c], sum);
+      for (int k = 0; k < kr; ++k) sum = fmaf(zk[t * r + k], bk[k * d + c], sum);
       kv[t * (d + 1) + c] = sum;
     }
     __syncthreads();
@@ -141,13 +153,16 @@ __global__ void __launch_bounds__(kSimtThreads) lrkv_split_simt(SplitArgs a) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
       if (lane == 0) sc[gi * T + t] = (t < n) ? dot * a.scale_log2 : -CUDART_INF_F;
+      if (ADAPT && lane == 0 && t < n)
+        ad.scores[((size_t)b * a.Hq + (size_t)g * G + gi) * a.Lcap + t0 + t] = dot * a.scale_log2;
     }
     __syncthreads();
     // rebuilt value tile V = Z_V B_V (overwrites the key tile)
     for (int i = tid; i < T * d; i += kSimtThreads) {
       const int t = i / d, c = i - t * d;
+      const int kr = ADAPT ? rk[t] : r;
       float sum = 0.f;
-      for (int k = 0; k < r; ++k) sum = fmaf(zv[t * r + k], bv[k * d + c], sum);
+      for (int k = 0; k < kr; ++k) sum = fmaf(zv[t * r + k], bv[k * d + c], sum);
       kv[t * (d + 1) + c] = sum;
     }
     // online softmax, one thread per query head
@@ -186,6 +201,36 @@ __global__ void __launch_bounds__(kSimtThreads) lrkv_split_simt(SplitArgs a) {
     const size_t h = (size_t)g * G + tid;
     a.lse_part[((size_t)b * a.Hq + h) * a.S + s] = (ms[tid] + log2f(ls[tid])) * CUDART_LN2_F;
   }
+}
+
+__global__ void __launch_bounds__(kSimtThreads) lrkv_split_simt(SplitArgs a) {
+  split_simt_body<false>(a, AdaptArgs{});
+}
+
+__global__ void __launch_bounds__(kSimtThreads) lrkv_split_simt_adaptive(SplitArgs a, AdaptArgs ad) {
+  split_simt_body<true>(a, ad);
+}
+
+// grid (ceil(max_seqlen / 256), Hkv, B), 256 threads: for every attended token of row
+// b and KV head g, the attention mass (the softmax weights of the group's G query
+// heads, from the kept log2 scores and the merged natural-log LSE) and the moving
+// average importance = beta * importance + (1 - beta) * mass. Launched after the
+// merge as a programmatic dependent: it waits for the merge (and so the split) first.
+__global__ void __launch_bounds__(256) lrkv_mass_ema(MassArgs m) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int t = blockIdx.x * 256 + threadIdx.x;
+  const int L = checked_len(m.seqlens, b, m.Lcap, m.max_seqlen, m.header, false);
+  if (t >= L) return;
+  const int G = m.Hq / m.Hkv;
+  float mass = 0.f;
+  for (int gi = 0; gi < G; ++gi) {
+    const size_t h = (size_t)b * m.Hq + (size_t)g * G + gi;
+    mass += exp2f(m.scores[h * m.Lcap + t] - m.lse[h] * CUDART_L2E_F);
+  }
+  float* p = m.imp + ((size_t)b * m.Hkv + g) * m.Lcap + t;
+  *p = m.beta * *p + (1.f - m.beta) * mass;
 }
 
 // grid (B * Hq), 128 threads (one per output dimension, d <= 128), S floats of dynamic
@@ -728,7 +773,7 @@ __global__ void __launch_bounds__(kProjThreads, 2) lrkv_project_append_kernel(Pr
 size_t simt_smem_bytes(int r, int d, int G) {
   const int T = kSimtTile;
   return sizeof(float) * ((size_t)2 * r * d + 2 * (size_t)G * d + 2 * (size_t)T * r +
-                          (size_t)T * (d + 1) + (size_t)G * T + 3 * (size_t)G);
+                          (size_t)T * (d + 1) + (size_t)G * T + 3 * (size_t)G + (size_t)T);
 }
 
 cudaError_t launch_split_simt(const SplitArgs& a, const Plan& p, cudaStream_t st) {
@@ -741,6 +786,24 @@ cudaError_t launch_split_simt(const SplitArgs& a, const Plan& p, cudaStream_t st
   }
   dim3 grid(a.S, a.Hkv, a.B);
   return launch_pdl(lrkv_split_simt, grid, dim3(kSimtThreads), (size_t)p.smem, st, a);
+}
+
+cudaError_t launch_split_simt_adaptive(const SplitArgs& a, const AdaptArgs& ad, const Plan& p,
+                                       cudaStream_t st) {
+  static int configured_smem = 0;
+  if (p.smem > configured_smem) {
+    cudaError_t e = cudaFuncSetAttribute(lrkv_split_simt_adaptive,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
+    if (e != cudaSuccess) return e;
+    configured_smem = p.smem;
+  }
+  dim3 grid(a.S, a.Hkv, a.B);
+  return launch_pdl(lrkv_split_simt_adaptive, grid, dim3(kSimtThreads), (size_t)p.smem, st, a, ad);
+}
+
+cudaError_t launch_mass_ema(const MassArgs& m, cudaStream_t st) {
+  const int tiles = std::max(1, (m.max_seqlen + 255) / 256);
+  return launch_pdl(lrkv_mass_ema, dim3(tiles, m.Hkv, m.B), dim3(256), 0, st, m);
 }
 
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st) {

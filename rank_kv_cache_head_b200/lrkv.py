@@ -81,6 +81,9 @@ def lib() -> ctypes.CDLL:
         L.lrkv_read_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
         L.lrkv_debug_stall_next_launch.argtypes = [ctypes.c_int32]
         L.lrkv_project_append.argtypes = [dp, ctypes.c_int32] + [_vp] * 9 + [ctypes.c_size_t, _vp]
+        L.lrkv_decode_attn_adaptive.argtypes = ([dp] + [_vp] * 9 + [ctypes.c_float, ctypes.c_int32,
+                                                 ctypes.c_float] + [_vp] * 4 +
+                                                [ctypes.c_size_t, _vp])
         _lib = L
     return _lib
 
@@ -175,6 +178,30 @@ def decode_attn(dims: Dims, q, ZK, ZV, ZK_scale, ZV_scale, BK, BV, seqlens, out,
     rc = lib().lrkv_decode_attn(ctypes.byref(dims), *args, workspace.numel(), _stream(stream))
     if rc:
         raise LrkvError("lrkv_decode_attn", rc)
+
+
+def decode_attn_adaptive(dims: Dims, q, ZK, ZV, ZK_scale, ZV_scale, BK, BV, seqlens,
+                         importance, tau, r_low, beta, scores, out, lse_out, workspace,
+                         stream=None) -> None:
+    """lrkv_decode_attn_adaptive: decode attention with tokens below the importance
+    threshold rebuilt at rank r_low, then importance <- beta * importance + (1 - beta) *
+    attention mass. importance [B][Hkv][max_seq] and scores [B][Hq][max_seq] fp32."""
+    sh = _shapes(dims)
+    n_imp = dims.batch * dims.n_kv_heads * dims.max_seq
+    n_sc = dims.batch * dims.n_q_heads * dims.max_seq
+    args = [
+        _ptr(q, "q", *sh["q"][::-1]), _ptr(ZK, "ZK", *sh["Z"][::-1]), _ptr(ZV, "ZV", *sh["Z"][::-1]),
+        _ptr(ZK_scale, "ZK_scale", *sh["S"][::-1]), _ptr(ZV_scale, "ZV_scale", *sh["S"][::-1]),
+        _ptr(BK, "BK", *sh["B"][::-1]), _ptr(BV, "BV", *sh["B"][::-1]),
+        _ptr(seqlens, "seqlens", *sh["seq"][::-1]),
+        _ptr(importance, "importance", (torch.float32,), n_imp)]
+    rc = lib().lrkv_decode_attn_adaptive(
+        ctypes.byref(dims), *args, float(tau), int(r_low), float(beta),
+        _ptr(scores, "scores", (torch.float32,), n_sc), _ptr(out, "out", *sh["q"][::-1]),
+        _ptr(lse_out, "lse_out", *sh["lse"][::-1]), _ptr(workspace, "workspace"),
+        workspace.numel(), _stream(stream))
+    if rc:
+        raise LrkvError("lrkv_decode_attn_adaptive", rc)
 
 
 def decode_attn_timed(dims: Dims, q, ZK, ZV, ZK_scale, ZV_scale, BK, BV, seqlens, out,

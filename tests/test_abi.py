@@ -1,5 +1,5 @@
-"""CPU checks of the C ABI: the library loads, exports every function include/lrkv.h
-declares, and validates arguments (no compute call is made without a GPU)."""
+"""CPU checks of the C ABI: the library loads, exports every function the headers in
+include/ declare, and validates arguments (no compute call is made without a GPU)."""
 import ctypes
 import os
 import re
@@ -9,11 +9,12 @@ import pytest
 from rank_kv_cache_head_b200 import lrkv
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "lrkv.h")
+HEADERS = sorted(os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+                 if f.endswith(".h"))
 
 
 def declared_functions():
-    src = open(HEADER).read()
+    src = "".join(open(h).read() for h in HEADERS)
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(lrkv_[a-z_0-9]+)\s*\(", src)))
 
@@ -21,7 +22,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ("lrkv_decode_attn", "lrkv_append", "lrkv_workspace_bytes",
-                     "lrkv_read_status", "lrkv_strerror"):
+                     "lrkv_read_status", "lrkv_strerror", "lrkv_project_append",
+                     "lrkv_decode_attn_adaptive"):
         assert required in names
 
 
@@ -114,3 +116,25 @@ def test_binding_refuses_cpu_tensors():
     t = torch.zeros(4)
     with pytest.raises((ValueError, TypeError)):
         lrkv.decode_attn(d, t, t, t, None, None, t, t, t, t, t)
+
+
+def test_adaptive_arguments_checked_before_any_launch():
+    """lrkv_decode_attn_adaptive refuses the tensor-core kernel, NULL state buffers and
+    out-of-range rank or decay before touching the device."""
+    L = lrkv.lib()
+    d = _dims()
+    fake = ctypes.c_void_p(16)
+
+    def call(dims, imp=fake, scores=fake, lse=fake, r_low=8, beta=0.5):
+        return L.lrkv_decode_attn_adaptive(ctypes.byref(dims), fake, fake, fake, None, None, fake,
+                                           fake, fake, imp, 0.5, r_low, beta, scores, fake, lse,
+                                           fake, 1 << 20, None)
+    assert call(_dims(algo="tcgen05")) == -6
+    assert call(d, imp=None) == -7
+    assert call(d, scores=None) == -7
+    assert call(d, lse=None) == -7
+    assert call(d, r_low=0) == -7
+    assert call(d, r_low=33) == -7
+    assert call(d, beta=1.5) == -7
+    assert call(d, beta=float("nan")) == -7
+    assert call(_dims(rank=12)) == -1

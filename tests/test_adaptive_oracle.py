@@ -153,3 +153,11 @@ def test_planted_mistakes_fail_the_loop_pin():
                     ema=lambda old, m, beta: (1 - beta) * old + beta * m)
     assert not np.allclose(got[0], inverted[0], atol=1e-6)
     assert not np.allclose(got[3], swapped[2], atol=1e-6)
+
+
+def test_inputs_are_left_as_given():
+    q, ZK, ZV, BK, BV, seq, imp, _, _ = _case(40)
+    keep = [a.copy() for a in (q, ZK, ZV, BK, BV, imp)]
+    orc.decode_attention_adaptive(q, ZK, ZV, BK, BV, seq, imp, 0.5, 2, 0.7)
+    for a, b in zip((q, ZK, ZV, BK, BV, imp), keep):
+        np.testing.assert_array_equal(a, b)
