@@ -257,6 +257,46 @@ def decode_attention_adaptive(q, ZK, ZV, BK, BV, seqlens, importance, tau: float
     return out, lse, mass, new_imp
 
 
+def decode_attention_shared(q, ZK, ZV, DK, DV, seqlens, n_kv_heads: int, ZK_scale=None,
+                            ZV_scale=None):
+    """Cross-head shared latent ("AttentionPack", Metodologia 2.A, multi-head
+    compression: the key (value) rows of all heads are concatenated along the head axis
+    and factored once, so a token keeps one latent of rank R for every head and one
+    decompression matrix of R x (H d) serves them all).
+
+    q [B][Hq][d]; ZK, ZV [B][L_cap][R] (decoded codes); scales [B][L_cap] or None;
+    DK, DV [R][n_kv_heads * d]; seqlens [B]. KV head g's keys are Z_K D_K[:, g d:(g+1) d]
+    (its values likewise); query head h reads KV head h // G. Returns out [B][Hq][d] and
+    lse [B][Hq]. Reading: the concatenation order is head-major (head g owns columns
+    g d .. g d + d - 1 of D)."""
+    q = np.asarray(q, np.float64)
+    B, Hq, d = q.shape
+    G = Hq // n_kv_heads
+    out = np.zeros((B, Hq, d))
+    lse = np.full((B, Hq), -np.inf)
+    for b in range(B):
+        Lb = int(seqlens[b])
+        if Lb == 0:
+            continue
+        sk = None if ZK_scale is None else ZK_scale[b, :Lb]
+        sv = None if ZV_scale is None else ZV_scale[b, :Lb]
+        Zk = dequantise(np.asarray(ZK[b, :Lb, :], np.float64), sk)
+        Zv = dequantise(np.asarray(ZV[b, :Lb, :], np.float64), sv)
+        Kall = Zk @ np.asarray(DK, np.float64)        # Lb x (H d): every head at once
+        Vall = Zv @ np.asarray(DV, np.float64)
+        for h in range(Hq):
+            g = h // G
+            K = Kall[:, g * d:(g + 1) * d]
+            V = Vall[:, g * d:(g + 1) * d]
+            s = (K @ q[b, h]) / math.sqrt(d)
+            m = s.max()
+            e = np.exp(s - m)
+            l = e.sum()
+            out[b, h] = (e / l) @ V
+            lse[b, h] = m + math.log(l)
+    return out, lse
+
+
 def decode_attention_reassociated(q, ZK, ZV, BK, BV, seqlens, ZK_scale=None, ZV_scale=None):
     """The same attention computed without rebuilding K, V: scores as
     (q B_K^T) Z_K^T and output as (p Z_V) B_V. Exactly equal in real arithmetic;
