@@ -70,6 +70,9 @@ def parse():
     ap.add_argument("--adaptive-rlow", type=int, default=0, metavar="R",
                     help="also time the attention-aware partial decompression with tokens "
                          "below the importance threshold rebuilt at rank R (0: skip)")
+    ap.add_argument("--shared-rank", type=int, default=0, metavar="R",
+                    help="also time decode attention over a cross-head shared latent of rank "
+                         "R on this workload's shape (0: skip)")
     ap.add_argument("--n-visual", type=int, default=0, metavar="P",
                     help="modality-separated factors: positions < P use a visual factor "
                          "set, the rest a text set (0: one set, the default)")
@@ -388,6 +391,58 @@ def measure_adaptive(wl, dev, r_low: int, tau: float = 0.5, beta: float = 0.9):
             "launches": f"CUDA graph of {per_graph} calls, one cache copy"}
 
 
+def measure_shared(wl, dev, R: int):
+    """Time lrkv_decode_attn_shared (cross-head shared latent, CUDA-core kernel) on this
+    workload's batch, heads and lengths with one rank-R latent row per token for every
+    KV head (bf16 latents and decompression matrices, seeded). Returns a dict."""
+    target = seqlens_for(wl)
+    cap = ((int(target.max()) + 7) // 8) * 8
+    g = torch.Generator(device="cpu").manual_seed(wl.seed + 55)
+    io_t = torch.float32 if wl.io_dtype == "f32" else torch.bfloat16
+    B, Hq, Hkv, d = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.d_head
+    q = torch.randn(B, Hq, d, generator=g).to(io_t).to(dev)
+    ZK = torch.randn(B, cap, R, generator=g).to(io_t).to(dev)
+    ZV = torch.randn(B, cap, R, generator=g).to(io_t).to(dev)
+    DK = (torch.randn(R, Hkv * d, generator=g) / math.sqrt(R)).to(io_t).to(dev)
+    DV = (torch.randn(R, Hkv * d, generator=g) / math.sqrt(R)).to(io_t).to(dev)
+    seq = torch.from_numpy(target.astype(np.int32)).to(dev)
+    dims = lrkv.make_dims(B, Hq, Hkv, d, R, cap, int(target.max()), wl.io_dtype, wl.io_dtype, 0,
+                          "simt")
+    out = torch.empty_like(q)
+    ws = lrkv.new_workspace(dims, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    per_graph, replays = 10, 3
+    with torch.cuda.stream(stream):
+        call = lambda: lrkv.decode_attn_shared(dims, q, ZK, ZV, None, None, DK, DV, seq, out, ws,
+                                               stream=stream)
+        for _ in range(3):
+            call()
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for _ in range(per_graph):
+                call()
+        graph.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(replays):
+            graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (per_graph * replays)
+    st = lrkv.read_status(ws)
+    if st:
+        raise RuntimeError(f"device status {st} after the shared-latent timing")
+    lat = int(target.sum()) * 2 * R * ZK.element_size()
+    peak, kind = peaks()
+    return {"kernel": "CUDA-core split (simt, shared-latent layout) + merge", "rank": R,
+            "latent_bytes_per_token": 2 * R * ZK.element_size(),
+            "per_head_equivalent_bytes_per_token": 2 * wl.rank * Hkv * ZK.element_size(),
+            "us_per_call": us, "latent_GBs": lat / (us * 1e-6) / 1e9, "peak_GBs": peak,
+            "peak_kind": kind, "frac": lat / (us * 1e-6) / 1e9 / peak,
+            "launches": f"CUDA graph of {per_graph} calls"}
+
+
 def run_ours(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -592,6 +647,8 @@ def run_ours(args, rank, world, local):
         line["project_append"] = measure_projection(wl, dev, args.projection_dmodel)
     if rank == 0 and args.adaptive_rlow > 0:
         line["adaptive"] = measure_adaptive(wl, dev, args.adaptive_rlow)
+    if rank == 0 and args.shared_rank > 0:
+        line["shared_latent"] = measure_shared(wl, dev, args.shared_rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         per_unit, n, lb, spent = oracle_sample(wl, inputs, args.cpu_seconds, n_visual=args.n_visual)
         cores = blas_threads()

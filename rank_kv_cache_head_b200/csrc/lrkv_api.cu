@@ -12,9 +12,10 @@
 #include <tuple>
 #include <vector>
 
-#include "lrkv_adaptive_internal.h"
+#include "lrkv_ext_internal.h"
 #include "lrkv_internal.h"
 #include "lrkv_adaptive.h"
+#include "lrkv_shared.h"
 
 namespace lrkv {
 
@@ -239,11 +240,11 @@ static int decode_impl(const lrkv_dims* dims, const void* q, const void* ZK, con
                        const void* BV, const int32_t* seqlens, void* out, float* lse_out,
                        void* workspace, size_t workspace_bytes, void* stream,
                        void* ev_split_begin, void* ev_split_end, const AdaptArgs* ad,
-                       float beta) {
+                       float beta, bool shared = false) {
   Plan p;
   int rc = make_plan(dims, &p);
   if (rc) return rc;
-  if (ad && p.algo != LRKV_ALGO_SIMT) return LRKV_ERR_UNSUPPORTED;
+  if ((ad || shared) && p.algo != LRKV_ALGO_SIMT) return LRKV_ERR_UNSUPPORTED;
   const bool quant = dims->latent_dtype == LRKV_I8 || dims->latent_dtype == LRKV_E4M3;
   if (!q || !ZK || !ZV || !BK || !BV || !seqlens || !out || !workspace) return LRKV_ERR_ARG;
   if (quant != (ZK_scale != nullptr) || quant != (ZV_scale != nullptr)) return LRKV_ERR_ARG;
@@ -299,9 +300,10 @@ static int decode_impl(const lrkv_dims* dims, const void* q, const void* ZK, con
     a.device_chunk = p.device_chunk;
   }
   record_event(ev_split_begin, st);
-  cudaError_t e = ad ? launch_split_simt_adaptive(a, *ad, p, st)
-                     : (p.algo == LRKV_ALGO_TCGEN05) ? launch_split_tc(a, p, st)
-                                                     : launch_split_simt(a, p, st);
+  cudaError_t e = ad       ? launch_split_simt_adaptive(a, *ad, p, st)
+                  : shared ? launch_split_simt_shared(a, p, st)
+                  : (p.algo == LRKV_ALGO_TCGEN05) ? launch_split_tc(a, p, st)
+                                                  : launch_split_simt(a, p, st);
   if (e != cudaSuccess) return LRKV_ERR_LAUNCH;
   record_event(ev_split_end, st);
 
@@ -349,6 +351,21 @@ int lrkv_decode_attn_timed(const lrkv_dims* dims, const void* q, const void* ZK,
   return decode_impl(dims, q, ZK, ZV, ZK_scale, ZV_scale, BK, BV, seqlens, out, lse_out,
                      workspace, workspace_bytes, stream, ev_split_begin, ev_split_end, nullptr,
                      0.f);
+}
+
+int lrkv_decode_attn_shared(const lrkv_dims* dims, const void* q, const void* ZK,
+                            const void* ZV, const float* ZK_scale, const float* ZV_scale,
+                            const void* DK, const void* DV, const int32_t* seqlens, void* out,
+                            float* lse_out, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (dims->algo == LRKV_ALGO_TCGEN05) return LRKV_ERR_UNSUPPORTED;
+  if (dims->n_visual != 0) return LRKV_ERR_DIMS;
+  lrkv_dims d = *dims;
+  d.algo = LRKV_ALGO_SIMT;
+  return decode_impl(&d, q, ZK, ZV, ZK_scale, ZV_scale, DK, DV, seqlens, out, lse_out,
+                     workspace, workspace_bytes, stream, nullptr, nullptr, nullptr, 0.f, true);
 }
 
 int lrkv_decode_attn_adaptive(const lrkv_dims* dims, const void* q, const void* ZK,

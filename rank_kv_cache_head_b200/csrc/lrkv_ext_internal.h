@@ -1,5 +1,7 @@
-// Internal declarations of the attention-aware partial decompression (the CUDA-core
-// split kernel with a per-token rank, and the attention-mass moving average).
+// Internal declarations of the CUDA-core decode variants beyond the per-head cache:
+// the attention-aware partial decompression (a per-token rank, and the attention-mass
+// moving average) and the cross-head shared latent (one latent per token for every KV
+// head, one decompression matrix).
 #pragma once
 
 #include "lrkv_internal.h"
@@ -28,5 +30,8 @@ struct MassArgs {
 cudaError_t launch_split_simt_adaptive(const SplitArgs& a, const AdaptArgs& ad, const Plan& p,
                                        cudaStream_t st);
 cudaError_t launch_mass_ema(const MassArgs& m, cudaStream_t st);
+// Shared latent: ZK/ZV [B][Lcap][r] and scales [B][Lcap]; BK/BV hold the decompression
+// matrices [r][Hkv * d] (KV head g owns columns g d .. g d + d - 1).
+cudaError_t launch_split_simt_shared(const SplitArgs& a, const Plan& p, cudaStream_t st);
 
 }  // namespace lrkv

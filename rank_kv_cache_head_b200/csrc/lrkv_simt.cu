@@ -15,7 +15,7 @@
 #include <cuda_fp8.h>
 #include <math_constants.h>
 
-#include "lrkv_adaptive_internal.h"
+#include "lrkv_ext_internal.h"
 #include "lrkv_internal.h"
 #include "lrkv_sm100.cuh"
 
@@ -68,7 +68,10 @@ __device__ __forceinline__ int checked_len(const int32_t* seqlens, int b, int Lc
 // ad.tau is rebuilt from its first ad.r_low latent components (the loop bound of the
 // reconstruction), and the scores of the attended tokens are kept for the moving
 // average of the attention mass.
-template <bool ADAPT>
+// SHARED: cross-head shared latent. The latents are [B][Lcap][r] (one row per token
+// for every KV head) and BK/BV the decompression matrices [r][Hkv * d], of which KV
+// head g uses columns g d .. g d + d - 1.
+template <bool ADAPT, bool SHARED>
 __device__ __forceinline__ void split_simt_body(const SplitArgs& a, const AdaptArgs& ad) {
   extern __shared__ float sm[];
   griddep_wait();
@@ -97,8 +100,13 @@ __device__ __forceinline__ void split_simt_body(const SplitArgs& a, const AdaptA
 
   const size_t fac_base = ((size_t)fset * a.Hkv + g) * r * d;   // factor set, then head
   for (int i = tid; i < r * d; i += kSimtThreads) {
-    bk[i] = load_io(a.BK, fac_base + i, a.io_dtype);
-    bv[i] = load_io(a.BV, fac_base + i, a.io_dtype);
+    size_t src = fac_base + i;
+    if (SHARED) {   // row k of the decompression matrix, this head's column block
+      const int k = i / d, c = i - k * d;
+      src = (size_t)k * a.Hkv * d + (size_t)g * d + c;
+    }
+    bk[i] = load_io(a.BK, src, a.io_dtype);
+    bv[i] = load_io(a.BV, src, a.io_dtype);
   }
   const size_t q_base = ((size_t)b * a.Hq + (size_t)g * G) * d;
   for (int i = tid; i < G * d; i += kSimtThreads) {
@@ -109,7 +117,8 @@ __device__ __forceinline__ void split_simt_body(const SplitArgs& a, const AdaptA
     ms[tid] = -CUDART_INF_F;
     ls[tid] = 0.f;
   }
-  const size_t row_base = ((size_t)b * a.Hkv + g) * (size_t)a.Lcap;  // token index base
+  // token index base: the (batch row, KV head) block, or the batch row's shared rows
+  const size_t row_base = SHARED ? (size_t)b * a.Lcap : ((size_t)b * a.Hkv + g) * (size_t)a.Lcap;
   const bool quant = a.latent_dtype == LRKV_I8 || a.latent_dtype == LRKV_E4M3;
 
   for (int t0 = t_begin; t0 < t_end; t0 += T) {
@@ -204,11 +213,15 @@ __device__ __forceinline__ void split_simt_body(const SplitArgs& a, const AdaptA
 }
 
 __global__ void __launch_bounds__(kSimtThreads) lrkv_split_simt(SplitArgs a) {
-  split_simt_body<false>(a, AdaptArgs{});
+  split_simt_body<false, false>(a, AdaptArgs{});
 }
 
 __global__ void __launch_bounds__(kSimtThreads) lrkv_split_simt_adaptive(SplitArgs a, AdaptArgs ad) {
-  split_simt_body<true>(a, ad);
+  split_simt_body<true, false>(a, ad);
+}
+
+__global__ void __launch_bounds__(kSimtThreads) lrkv_split_simt_shared(SplitArgs a) {
+  split_simt_body<false, true>(a, AdaptArgs{});
 }
 
 // grid (ceil(max_seqlen / 256), Hkv, B), 256 threads: for every attended token of row
@@ -799,6 +812,18 @@ cudaError_t launch_split_simt_adaptive(const SplitArgs& a, const AdaptArgs& ad, 
   }
   dim3 grid(a.S, a.Hkv, a.B);
   return launch_pdl(lrkv_split_simt_adaptive, grid, dim3(kSimtThreads), (size_t)p.smem, st, a, ad);
+}
+
+cudaError_t launch_split_simt_shared(const SplitArgs& a, const Plan& p, cudaStream_t st) {
+  static int configured_smem = 0;
+  if (p.smem > configured_smem) {
+    cudaError_t e = cudaFuncSetAttribute(lrkv_split_simt_shared,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem);
+    if (e != cudaSuccess) return e;
+    configured_smem = p.smem;
+  }
+  dim3 grid(a.S, a.Hkv, a.B);
+  return launch_pdl(lrkv_split_simt_shared, grid, dim3(kSimtThreads), (size_t)p.smem, st, a);
 }
 
 cudaError_t launch_mass_ema(const MassArgs& m, cudaStream_t st) {

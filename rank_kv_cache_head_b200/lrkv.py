@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
         L.lrkv_read_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
         L.lrkv_debug_stall_next_launch.argtypes = [ctypes.c_int32]
         L.lrkv_project_append.argtypes = [dp, ctypes.c_int32] + [_vp] * 9 + [ctypes.c_size_t, _vp]
+        L.lrkv_decode_attn_shared.argtypes = [dp] + [_vp] * 11 + [ctypes.c_size_t, _vp]
         L.lrkv_decode_attn_adaptive.argtypes = ([dp] + [_vp] * 9 + [ctypes.c_float, ctypes.c_int32,
                                                  ctypes.c_float] + [_vp] * 4 +
                                                 [ctypes.c_size_t, _vp])
@@ -178,6 +179,26 @@ def decode_attn(dims: Dims, q, ZK, ZV, ZK_scale, ZV_scale, BK, BV, seqlens, out,
     rc = lib().lrkv_decode_attn(ctypes.byref(dims), *args, workspace.numel(), _stream(stream))
     if rc:
         raise LrkvError("lrkv_decode_attn", rc)
+
+
+def decode_attn_shared(dims: Dims, q, ZK, ZV, ZK_scale, ZV_scale, DK, DV, seqlens, out,
+                       workspace, lse_out=None, stream=None) -> None:
+    """lrkv_decode_attn_shared: decode attention over a cross-head shared latent.
+    ZK/ZV [B][max_seq][rank], scales [B][max_seq], DK/DV [rank][n_kv_heads * d_head]."""
+    sh = _shapes(dims)
+    io = sh["q"][1]
+    nz = dims.batch * dims.max_seq * dims.rank
+    nd = dims.rank * dims.n_kv_heads * dims.d_head
+    ns = dims.batch * dims.max_seq
+    args = [
+        _ptr(q, "q", *sh["q"][::-1]), _ptr(ZK, "ZK", sh["Z"][1], nz), _ptr(ZV, "ZV", sh["Z"][1], nz),
+        _ptr(ZK_scale, "ZK_scale", (torch.float32,), ns), _ptr(ZV_scale, "ZV_scale", (torch.float32,), ns),
+        _ptr(DK, "DK", io, nd), _ptr(DV, "DV", io, nd),
+        _ptr(seqlens, "seqlens", *sh["seq"][::-1]), _ptr(out, "out", *sh["q"][::-1]),
+        _ptr(lse_out, "lse_out", *sh["lse"][::-1]), _ptr(workspace, "workspace")]
+    rc = lib().lrkv_decode_attn_shared(ctypes.byref(dims), *args, workspace.numel(), _stream(stream))
+    if rc:
+        raise LrkvError("lrkv_decode_attn_shared", rc)
 
 
 def decode_attn_adaptive(dims: Dims, q, ZK, ZV, ZK_scale, ZV_scale, BK, BV, seqlens,

@@ -23,7 +23,7 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ("lrkv_decode_attn", "lrkv_append", "lrkv_workspace_bytes",
                      "lrkv_read_status", "lrkv_strerror", "lrkv_project_append",
-                     "lrkv_decode_attn_adaptive"):
+                     "lrkv_decode_attn_adaptive", "lrkv_decode_attn_shared"):
         assert required in names
 
 
@@ -137,4 +137,16 @@ def test_adaptive_arguments_checked_before_any_launch():
     assert call(d, r_low=33) == -7
     assert call(d, beta=1.5) == -7
     assert call(d, beta=float("nan")) == -7
+    assert call(_dims(rank=12)) == -1
+
+
+def test_shared_latent_arguments_checked_before_any_launch():
+    L = lrkv.lib()
+    fake = ctypes.c_void_p(16)
+
+    def call(dims):
+        return L.lrkv_decode_attn_shared(ctypes.byref(dims), fake, fake, fake, None, None, fake,
+                                         fake, fake, fake, None, fake, 1 << 20, None)
+    assert call(_dims(algo="tcgen05")) == -6
+    assert call(_dims(n_visual=16)) == -1
     assert call(_dims(rank=12)) == -1
